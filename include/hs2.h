@@ -1,0 +1,177 @@
+/*
+ * hs2.h -- C ABI of a B200 (sm_100a) library for HySparse2's token-level
+ * KV Reuse hot path.
+ *
+ * The method (HySparse2 summary, onedev.kr/papers/146):
+ *   - "What differs": a full-attention layer computes exact attention and, per
+ *     query token, selects individual tokens: the recent-token window is always
+ *     taken first, then the highest-scoring tokens outside it.  The sparse
+ *     layers that follow reuse the selected tokens' KV entries.
+ *   - "How it works": inside a hybrid block the sparse layers reuse the full
+ *     layer's KV cache and selection indices unchanged (KV Reuse).
+ *   - "How to use": one shared KV head (MQA), no positional encoding in full
+ *     or sparse attention, W = 128 forced local tokens plus k = 1,024 global
+ *     tokens; efficiency quoted on an FP8 KV cache.
+ * Readings of what the page leaves open:
+ *   - score(t,s) = sum over the Hq query heads of softmax probability
+ *     exp(l_h(t,s) - lse_h(t)), l_h(t,s) = scale * <q_{t,h}, k_s>;
+ *   - window = positions max(0,t-W+1)..t (the query itself included);
+ *   - global candidates = positions 0..t-W; the k best by (score descending,
+ *     position ascending); all of them when there are at most k;
+ *   - the full layer's own output is full causal attention;
+ *   - decode: the new token sits at position T-1 of a cache of length T that
+ *     already holds its K/V;
+ *   - FP8 KV: x = scale_row * e4m3(code), one fp32 scale per token for K and
+ *     one for V.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers, row-major, last dim contiguous,
+ *     16-byte aligned.  The caller owns every buffer; the library allocates,
+ *     frees and synchronises nothing (hs2_get_last_device_error excepted).
+ *   - Every call is asynchronous on `stream`.  Arguments are validated on the
+ *     host before anything is launched; on failure a non-zero status is
+ *     returned and no kernel runs.  Launch failures map to HS2_ERR_CUDA.
+ *   - Supported: head dim d in {64, 128}; Hq in {4, 8, 16} query heads sharing
+ *     one KV head; W >= 1, k >= 0, W + k <= 2048; scale finite and > 0.
+ *   - Index output format (`idx`, W+k int32 per query): the window positions
+ *     ascending first, then the global picks in no particular order, then -1
+ *     padding.  |selection| = min(t+1, W+k).  Treat it as a set.
+ *   - Device-side data checks (decode lengths outside [1, Tmax], a query value
+ *     beyond the fp16 range +-65504 on an e4m3 path, an index outside [0, t])
+ *     do not fault: the kernel skips the offending work and records a flag that
+ *     hs2_get_last_device_error reports as HS2_ERR_DEVICE_DATA.
+ */
+#ifndef HS2_H
+#define HS2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st* hs2_stream_t;
+
+typedef enum {
+    HS2_OK = 0,
+    HS2_ERR_INVALID_ARG = 1,  /* null / misaligned pointer, bad size, bad scale */
+    HS2_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d, Hq, W+k, dtype) */
+    HS2_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace() size */
+    HS2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+    HS2_ERR_DEVICE_DATA = 5   /* a kernel met out-of-contract data (see above) */
+} hs2_status;
+
+typedef enum { HS2_KV_BF16 = 0, HS2_KV_E4M3 = 1 } hs2_kv_dtype;
+
+/* Prefill shape: B sequences of L tokens, Hq query heads, one KV head. */
+typedef struct {
+    int B, L, Hq, d, W, k;
+    float scale; /* softmax scale, normally 1/sqrt(d) */
+} hs2_prefill_shape;
+
+/* Decode shape: B sequences, caches of Tmax rows, one query token each. */
+typedef struct {
+    int B, Tmax, Hq, d, W, k;
+    float scale;
+    hs2_kv_dtype kv;
+} hs2_decode_shape;
+
+/* Human-readable name of a status code (static string). */
+const char* hs2_status_string(hs2_status s);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int hs2_version(void);
+
+/*
+ * Bytes of device workspace hs2_full_attn_select needs for `shape`
+ * (0 for an invalid shape).  Per query row it holds a candidate buffer of
+ * 2k+256 (score, position) entries plus the row's running threshold and count.
+ */
+size_t hs2_full_attn_select_workspace(const hs2_prefill_shape* shape);
+
+/*
+ * Full-attention layer with token selection (prefill).
+ * Defined by the "What differs" section of the HySparse2 summary: exact causal
+ * attention whose scores select, per query token, the window plus the top-k
+ * older tokens.
+ *   q   [B, L, Hq, d] bf16      queries
+ *   k,v [B, L, d]     bf16      the layer's single KV head (the cache the sparse
+ *                               layers reuse)
+ *   o   [B, L, Hq, d] bf16      out: full causal attention output
+ *   lse [B, L, Hq]    fp32      out: natural-log log-sum-exp of the scaled
+ *                               logits per (token, head); may be NULL
+ *   idx [B, L, W+k]   int32     out: selection, format above
+ *   workspace: device buffer of at least hs2_full_attn_select_workspace()
+ *   bytes; contents need no initialisation and are garbage afterwards.
+ * Calls on the same workspace must not overlap in time.
+ */
+hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, const void* k,
+                                const void* v, void* o, float* lse, int32_t* idx,
+                                void* workspace, size_t workspace_bytes, hs2_stream_t stream);
+
+/*
+ * Sparse layer (prefill): each query token attends, with its own queries, only
+ * to the K/V rows its inherited index set names (KV Reuse, "How it works").
+ *   q   [B, L, Hq, d] bf16      this sparse layer's queries
+ *   k,v [B, L, d]               the full layer's cache: bf16, or e4m3 codes (one
+ *                               byte each) when kv == HS2_KV_E4M3
+ *   k_scale, v_scale [B, L] fp32  per-token scales for e4m3 (NULL for bf16)
+ *   idx [B, L, S] int32, S = shape->W + shape->k: per token a set of positions
+ *                               in [0, t], -1 entries ignored, no repeats
+ *   o   [B, L, Hq, d] bf16      out; a token whose set is empty gets zeros
+ * e4m3 additionally needs |q| <= 65504 and per-token scales <= 65504.
+ */
+hs2_status hs2_sparse_attn(const hs2_prefill_shape* shape, const void* q, const void* k,
+                           const void* v, hs2_kv_dtype kv, const float* k_scale,
+                           const float* v_scale, const int32_t* idx, void* o,
+                           hs2_stream_t stream);
+
+/*
+ * Bytes of device workspace hs2_decode_select needs (0 for an invalid shape).
+ */
+size_t hs2_decode_select_workspace(const hs2_decode_shape* shape);
+
+/*
+ * Decode full layer with selection: one new query per sequence at position
+ * t = lengths[b]-1; exact attention over cache rows 0..t and the same
+ * selection rule as the prefill call.  Split over the cache length (split-KV).
+ *   q        [B, Hq, d] bf16
+ *   k_cache, v_cache [B, Tmax, d]  e4m3 codes (kv == HS2_KV_E4M3) or bf16
+ *   k_scale, v_scale [B, Tmax] fp32 (e4m3 only; NULL for bf16)
+ *   lengths  [B] int32, device, each in [1, Tmax]
+ *   o        [B, Hq, d] bf16  out: full attention output
+ *   lse      [B, Hq] fp32     out, may be NULL
+ *   idx      [B, W+k] int32   out: selection, format above
+ *   workspace: >= hs2_decode_select_workspace() bytes, no initialisation
+ *   needed; calls on the same workspace must not overlap in time.
+ */
+hs2_status hs2_decode_select(const hs2_decode_shape* shape, const void* q, const void* k_cache,
+                             const void* v_cache, const float* k_scale, const float* v_scale,
+                             const int32_t* lengths, void* o, float* lse, int32_t* idx,
+                             void* workspace, size_t workspace_bytes, hs2_stream_t stream);
+
+/*
+ * Decode sparse layer: sequence b's query attends to the cache rows idx[b]
+ * names (KV Reuse of the decode selection).
+ *   q [B, Hq, d] bf16; caches/scales as hs2_decode_select; idx [B, W+k] int32
+ *   with entries in [0, lengths[b]-1] or -1; o [B, Hq, d] bf16 out.
+ */
+hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const void* k_cache,
+                             const void* v_cache, const float* k_scale, const float* v_scale,
+                             const int32_t* lengths, const int32_t* idx, void* o,
+                             hs2_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reports (and clears) the first error met since
+ * the last call: a CUDA error (HS2_ERR_CUDA) or a device-side data flag
+ * (HS2_ERR_DEVICE_DATA).  Returns HS2_OK when there is none.
+ */
+hs2_status hs2_get_last_device_error(hs2_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H */

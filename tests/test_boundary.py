@@ -1,0 +1,141 @@
+"""Host-side boundary tests of the C ABI (no GPU needed): the library loads,
+exports every entry point include/hs2.h declares, sizes workspaces, and
+rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import token_level_top_hs2_b200 as hs2
+from token_level_top_hs2_b200 import build as hs2_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    hs2_build.build()
+    return hs2.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "hs2.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(hs2_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_four_entry_points():
+    names = declared_functions()
+    for n in ["hs2_full_attn_select", "hs2_sparse_attn", "hs2_decode_select",
+              "hs2_decode_sparse"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported"
+    assert sorted(hs2.EXPORTED) == names
+
+
+def test_status_strings(lib):
+    for code in range(6):
+        assert hs2.status_string(code) != "unknown status"
+    assert hs2.status_string(99) == "unknown status"
+    assert lib.hs2_version() >= 100
+
+
+def test_workspace_sizes(lib):
+    s = hs2.prefill_shape(1, 131072, 16, 128, 128, 1024)
+    ws = hs2.hs2_full_attn_select_workspace(s)
+    # lse area + one (2k+256)-entry buffer of 8-byte keys per query row
+    assert ws >= 131072 * (2 * 1024 + 256) * 8
+    assert hs2.hs2_full_attn_select_workspace(hs2.prefill_shape(1, 10, 3, 128, 8, 8)) == 0
+    d = hs2.decode_shape(16, 262144, 16, 128, 128, 1024)
+    assert hs2.hs2_decode_select_workspace(d) > 16 * 1024 * 8
+    assert hs2.hs2_decode_select_workspace(hs2.decode_shape(1, 100, 16, 96, 8, 8)) == 0
+
+
+FAKE = 1 << 20  # 16-byte aligned non-null stand-ins: never dereferenced on failure
+
+
+def call_full(lib, shape, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, idx=FAKE, ws=FAKE,
+              ws_bytes=1 << 40):
+    return lib.hs2_full_attn_select(ctypes.byref(shape), q, k, v, o, lse, idx, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("fields,code", [
+    (dict(d=96), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(Hq=3), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(W=1024, k=1025), hs2.HS2_ERR_UNSUPPORTED),
+    (dict(W=0), hs2.HS2_ERR_INVALID_ARG),
+    (dict(k=-1), hs2.HS2_ERR_INVALID_ARG),
+    (dict(L=0), hs2.HS2_ERR_INVALID_ARG),
+    (dict(B=0), hs2.HS2_ERR_INVALID_ARG),
+    (dict(scale=0.0), hs2.HS2_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), hs2.HS2_ERR_INVALID_ARG),
+])
+def test_full_select_rejects_bad_shapes(lib, fields, code):
+    base = dict(B=1, L=64, Hq=16, d=128, W=8, k=8, scale=0.1)
+    base.update(fields)
+    s = hs2.PrefillShape(**base)
+    assert call_full(lib, s) == code
+
+
+def test_full_select_rejects_bad_pointers_and_workspace(lib):
+    s = hs2.prefill_shape(1, 64, 16, 128, 8, 8)
+    assert call_full(lib, s, q=None) == hs2.HS2_ERR_INVALID_ARG
+    assert call_full(lib, s, idx=None) == hs2.HS2_ERR_INVALID_ARG
+    assert call_full(lib, s, k=FAKE + 8) == hs2.HS2_ERR_INVALID_ARG
+    assert call_full(lib, s, lse=FAKE + 4) == hs2.HS2_ERR_INVALID_ARG
+    need = hs2.hs2_full_attn_select_workspace(s)
+    assert call_full(lib, s, ws_bytes=need - 1) == hs2.HS2_ERR_WORKSPACE
+    assert lib.hs2_full_attn_select(None, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 40,
+                                    None) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_sparse_rejects_bad_arguments(lib):
+    s = hs2.prefill_shape(1, 64, 16, 128, 8, 8)
+    f = lib.hs2_sparse_attn
+    assert f(ctypes.byref(s), FAKE, FAKE, FAKE, hs2.HS2_KV_E4M3, None, FAKE, FAKE, FAKE,
+             None) == hs2.HS2_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), FAKE, FAKE, FAKE, 7, None, None, FAKE, FAKE,
+             None) == hs2.HS2_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), FAKE, FAKE, FAKE, hs2.HS2_KV_BF16, None, None, None, FAKE,
+             None) == hs2.HS2_ERR_INVALID_ARG
+    s64 = hs2.prefill_shape(1, 64, 16, 64, 8, 8)
+    assert f(ctypes.byref(s64), FAKE, FAKE, FAKE, hs2.HS2_KV_E4M3, FAKE, FAKE, FAKE, FAKE,
+             None) == hs2.HS2_ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_arguments(lib):
+    s = hs2.decode_shape(2, 1000, 16, 128, 8, 8, "e4m3")
+    f = lib.hs2_decode_select
+    need = hs2.hs2_decode_select_workspace(s)
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE]
+    assert f(ctypes.byref(s), *args, need - 1, None) == hs2.HS2_ERR_WORKSPACE
+    bad = list(args)
+    bad[3] = None  # k_scale missing for e4m3
+    assert f(ctypes.byref(s), *bad, need, None) == hs2.HS2_ERR_INVALID_ARG
+    bad = list(args)
+    bad[5] = None  # lengths
+    assert f(ctypes.byref(s), *bad, need, None) == hs2.HS2_ERR_INVALID_ARG
+    s_bad = hs2.DecodeShape(2, 0, 16, 128, 8, 8, 0.1, 1)
+    assert f(ctypes.byref(s_bad), *args, need, None) == hs2.HS2_ERR_INVALID_ARG
+    s_kv = hs2.DecodeShape(2, 100, 16, 128, 8, 8, 0.1, 5)
+    assert f(ctypes.byref(s_kv), *args, need, None) == hs2.HS2_ERR_INVALID_ARG
+    g = lib.hs2_decode_sparse
+    assert g(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+             None) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = hs2._lib
+    hs2._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="not built"):
+            hs2.load(str(tmp_path / "missing.so"))
+    finally:
+        hs2._lib = saved

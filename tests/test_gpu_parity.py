@@ -1,0 +1,245 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Tolerances: max-abs 1e-2 on bf16 outputs with bf16 KV and 2e-2 with e4m3 KV;
+selections identical except for swaps whose oracle score lies within 1e-5
+(relative) of the oracle's k-th score; windows identical.  The sparse kernels
+are checked in isolation (fed the oracle's indices) and end to end (the
+oracle re-run on the GPU's indices).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity import check_selection, check_structure, max_abs
+from token_level_top_hs2_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 1e-2
+TOL_E4M3 = 2e-2
+TOL_LSE = 2e-3
+
+
+def cuda(x):
+    return x.cuda() if isinstance(x, torch.Tensor) else x
+
+
+def sample_rows(B, L, n, seed, seg=256):
+    """First 64, last 64, 64 at segment boundaries, the rest uniform; all b."""
+    g = np.random.default_rng(seed)
+    per = max(1, n // B)
+    rows = []
+    for b in range(B):
+        t = set(range(min(64, L)))
+        t |= set(range(max(0, L - 64), L))
+        bnd = np.arange(seg, L, seg)
+        if bnd.size:
+            t |= set(g.choice(bnd, size=min(64, bnd.size), replace=False).tolist())
+        rest = per - len(t)
+        if rest > 0:
+            t |= set(g.choice(L, size=min(rest, L), replace=False).tolist())
+        rows += [b * L + x for x in sorted(t)]
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+def run_full(hs2, x, rows=None):
+    o, lse, idx = hs2.hs2_full_attn_select(cuda(x.q), cuda(x.k_), cuda(x.v), x.W, x.k)
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == 0
+    B, L, Hq, d = x.q.shape
+    o = o.float().cpu().numpy().reshape(B * L, Hq, d)
+    lse = lse.cpu().numpy().reshape(B * L, Hq)
+    idx = idx.cpu().numpy().reshape(B * L, -1)
+    return o, lse, idx
+
+
+def check_full_layer(hs2, x, rows=None):
+    B, L = x.q.shape[:2]
+    o, lse, idx = run_full(hs2, x)
+    t_all = np.tile(np.arange(L), B)
+    check_structure(idx, t_all, x.W, x.k)
+    if rows is None:
+        rows = np.arange(B * L, dtype=np.int64)
+    ora = oracle.full_select(x.q, x.k_, x.v, x.W, x.k, rows=rows, probe=idx[rows])
+    assert max_abs(o[rows], ora["o"]) <= TOL_BF16
+    assert max_abs(lse[rows], ora["lse"]) <= TOL_LSE
+    n_swap, overlap = check_selection(idx[rows], ora, rows % L, x.W, x.k)
+    return o, idx, ora, rows, n_swap, overlap
+
+
+@pytest.mark.parametrize("shape", [
+    dict(B=1, L=1024, Hq=4, d=64, W=32, k=128, n_topics=8, seg=128),   # the tiny prefill
+    dict(B=2, L=777, Hq=16, d=128, W=128, k=256, n_topics=8, seg=256),  # ragged tail, B=2
+    dict(B=1, L=300, Hq=8, d=128, W=16, k=0, n_topics=4, seg=64),       # window only
+    dict(B=1, L=5, Hq=16, d=64, W=4, k=8, n_topics=2, seg=4),           # shorter than a tile
+])
+def test_full_attn_select_matches_oracle(cuda_lib, shape):
+    s = dict(shape)
+    x = inputs.make_prefill(seed=inputs.seed_for(0, 1), n_sparse=1, **s)
+    _, idx, ora, rows, n_swap, overlap = check_full_layer(cuda_lib, x)
+    assert overlap > 0.999
+
+
+def test_full_attn_select_ties_take_lower_index(cuda_lib):
+    """Keys drawn from 4 distinct rows: many exact score ties straddle the cut."""
+    B, L, Hq, d, W, k = 1, 640, 16, 128, 16, 40
+    g = torch.Generator().manual_seed(3)
+    q = torch.randn(B, L, Hq, d, generator=g).bfloat16()
+    base = torch.randn(4, d, generator=g)
+    k_ = base[torch.randint(0, 4, (L,), generator=g)].unsqueeze(0).bfloat16()
+    v = torch.randn(B, L, d, generator=g).bfloat16()
+    x = inputs.PrefillInputs(B, L, Hq, d, W, k, q, k_, v, [], None, None, None)
+    o, lse, idx = run_full(cuda_lib, x)
+    ora = oracle.full_select(q, k_, v, W, k, probe=idx)
+    n_swap, _ = check_selection(idx, ora, np.arange(L), W, k, rel=1e-5)
+    assert max_abs(o, ora["o"]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_sparse_attn_isolated_and_end_to_end(cuda_lib, kv):
+    B, L, Hq, d, W, k = 2, 900, 16, 128, 64, 192
+    x = inputs.make_prefill(B, L, Hq, d, W, k, n_topics=8, seg=128, n_sparse=1,
+                            seed=inputs.seed_for(0, 2))
+    if kv == "e4m3":
+        kc, ks = inputs.quantize_e4m3_per_token(x.k_)
+        vc, vs = inputs.quantize_e4m3_per_token(x.v)
+    else:
+        kc, vc, ks, vs = x.k_, x.v, None, None
+    ora_sel = oracle.full_select(x.q, x.k_, x.v, W, k)
+    idx_ora = torch.from_numpy(ora_sel["idx"]).reshape(B, L, W + k)
+    qs = x.q_sparse[0]
+    # isolation: oracle indices
+    o = cuda_lib.hs2_sparse_attn(cuda(qs), cuda(kc), cuda(vc), cuda(idx_ora), kv=kv,
+                                 k_scale=cuda(ks), v_scale=cuda(vs), W=W, k_top=k)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    ref = oracle.sparse(qs, kc, vc, idx_ora, kv=kv, k_scale=ks, v_scale=vs)
+    tol = TOL_E4M3 if kv == "e4m3" else TOL_BF16
+    assert max_abs(o.float().cpu().numpy().reshape(B * L, Hq, d), ref) <= tol
+    # end to end: GPU selection feeding the GPU sparse layer, oracle on the GPU's indices
+    _, _, idx_gpu = cuda_lib.hs2_full_attn_select(cuda(x.q), cuda(x.k_), cuda(x.v), W, k)
+    o2 = cuda_lib.hs2_sparse_attn(cuda(qs), cuda(kc), cuda(vc), idx_gpu, kv=kv,
+                                  k_scale=cuda(ks), v_scale=cuda(vs), W=W, k_top=k)
+    ref2 = oracle.sparse(qs, kc, vc, idx_gpu.cpu(), kv=kv, k_scale=ks, v_scale=vs)
+    assert max_abs(o2.float().cpu().numpy().reshape(B * L, Hq, d), ref2) <= tol
+
+
+def test_sparse_equals_full_when_budget_covers(cuda_lib):
+    """W+k >= L selects everything: the sparse layer with the full layer's own
+    queries must reproduce the full layer's output."""
+    B, L, Hq, d, W, k = 1, 200, 16, 128, 8, 200
+    x = inputs.make_prefill(B, L, Hq, d, W, k, seed=5)
+    o, _, idx = cuda_lib.hs2_full_attn_select(cuda(x.q), cuda(x.k_), cuda(x.v), W, k)
+    o2 = cuda_lib.hs2_sparse_attn(cuda(x.q), cuda(x.k_), cuda(x.v), idx, W=W, k_top=k)
+    torch.cuda.synchronize()
+    assert (o.float() - o2.float()).abs().max().item() <= TOL_BF16
+
+
+def test_sparse_attn_flags_out_of_range_indices(cuda_lib):
+    B, L, Hq, d = 1, 64, 16, 128
+    x = inputs.make_prefill(B, L, Hq, d, 4, 4, seed=6)
+    idx = torch.full((B, L, 8), -1, dtype=torch.int32)
+    idx[0, :, 0] = torch.arange(L)
+    idx[0, 10, 1] = 11  # beyond t = 10
+    cuda_lib.hs2_sparse_attn(cuda(x.q), cuda(x.k_), cuda(x.v), cuda(idx), W=4, k_top=4)
+    assert cuda_lib.hs2_get_last_device_error() == cuda_lib.HS2_ERR_DEVICE_DATA
+    assert cuda_lib.hs2_get_last_device_error() == 0  # cleared
+
+
+def _decode_case(kv, B, T, Hq, d, W, k, lengths=None, seed=0):
+    return inputs.make_decode(B, T, Hq, d, W, k, kv=kv, seed=seed, lengths=lengths,
+                              n_needles=16, n_sparse=1)
+
+
+def run_decode(hs2, x):
+    o, lse, idx = hs2.hs2_decode_select(cuda(x.q), cuda(x.k_cache), cuda(x.v_cache),
+                                        cuda(x.lengths), x.W, x.k, kv=x.kv,
+                                        k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale))
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == 0
+    return o.float().cpu().numpy(), lse.cpu().numpy(), idx.cpu().numpy()
+
+
+@pytest.mark.parametrize("kv,B,T,Hq,d,W,k,lengths", [
+    ("e4m3", 3, 20000, 16, 128, 128, 1024, [20000, 9000, 1100]),
+    ("e4m3", 2, 70000, 16, 128, 128, 1024, None),     # several merge groups
+    ("bf16", 2, 5000, 8, 64, 32, 128, [5000, 77]),
+    ("e4m3", 4, 300, 4, 128, 16, 0, [300, 1, 17, 250]),  # window only, length 1
+])
+def test_decode_select_matches_oracle(cuda_lib, kv, B, T, Hq, d, W, k, lengths):
+    x = _decode_case(kv, B, T, Hq, d, W, k, lengths, seed=inputs.seed_for(3, 7))
+    o, lse, idx = run_decode(cuda_lib, x)
+    ora = oracle.decode_select(x.q, x.k_cache, x.v_cache, x.lengths, W, k, kv=kv,
+                               k_scale=x.k_scale, v_scale=x.v_scale, probe=idx)
+    tol = TOL_E4M3 if kv == "e4m3" else TOL_BF16
+    assert max_abs(o, ora["o"]) <= tol
+    assert max_abs(lse, ora["lse"]) <= TOL_LSE
+    t = x.lengths.numpy().astype(np.int64) - 1
+    check_structure(idx, t, W, k)
+    check_selection(idx, ora, t, W, k)
+
+
+@pytest.mark.parametrize("kv", ["e4m3", "bf16"])
+def test_decode_sparse_isolated_and_end_to_end(cuda_lib, kv):
+    B, T, Hq, d, W, k = 5, 12000, 16, 128, 128, 1024
+    x = _decode_case(kv, B, T, Hq, d, W, k, [12000, 5000, 1152, 1000, 3], seed=11)
+    ora = oracle.decode_select(x.q, x.k_cache, x.v_cache, x.lengths, W, k, kv=kv,
+                               k_scale=x.k_scale, v_scale=x.v_scale)
+    idx_ora = torch.from_numpy(ora["idx"])
+    qs = x.q_sparse[0]
+    o = cuda_lib.hs2_decode_sparse(cuda(qs), cuda(x.k_cache), cuda(x.v_cache), cuda(x.lengths),
+                                   cuda(idx_ora), kv=kv, k_scale=cuda(x.k_scale),
+                                   v_scale=cuda(x.v_scale), W=W, k_top=k)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    ref = oracle.decode_sparse(qs, x.k_cache, x.v_cache, idx_ora, kv=kv, k_scale=x.k_scale,
+                               v_scale=x.v_scale)
+    tol = TOL_E4M3 if kv == "e4m3" else TOL_BF16
+    assert max_abs(o.float().cpu().numpy(), ref) <= tol
+    _, _, idx_gpu = run_decode(cuda_lib, x)
+    o2 = cuda_lib.hs2_decode_sparse(cuda(qs), cuda(x.k_cache), cuda(x.v_cache), cuda(x.lengths),
+                                    cuda(torch.from_numpy(idx_gpu)), kv=kv,
+                                    k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale), W=W,
+                                    k_top=k)
+    ref2 = oracle.decode_sparse(qs, x.k_cache, x.v_cache, idx_gpu, kv=kv, k_scale=x.k_scale,
+                                v_scale=x.v_scale)
+    assert max_abs(o2.float().cpu().numpy(), ref2) <= tol
+
+
+def test_decode_flags_bad_length(cuda_lib):
+    x = _decode_case("e4m3", 2, 1000, 16, 128, 16, 32, seed=2)
+    x.lengths[1] = 2000  # beyond Tmax
+    o, lse, idx = cuda_lib.hs2_decode_select(cuda(x.q), cuda(x.k_cache), cuda(x.v_cache),
+                                             cuda(x.lengths), 16, 32, kv="e4m3",
+                                             k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale))
+    assert cuda_lib.hs2_get_last_device_error() == cuda_lib.HS2_ERR_DEVICE_DATA
+    assert (idx[1] == -1).all().item()
+
+
+def test_e4m3_subnormal_codes_are_exact(cuda_lib):
+    """Caches made only of subnormal and tiny normal e4m3 codes."""
+    B, T, Hq, d, W, k = 1, 64, 16, 128, 8, 16
+    g = torch.Generator().manual_seed(4)
+    codes = torch.randint(0, 16, (B, T, d), generator=g).to(torch.uint8)  # exp field 0..1
+    codes |= (torch.randint(0, 2, (B, T, d), generator=g).to(torch.uint8) << 7)
+    kc = codes.clone()
+    vc = torch.roll(codes, 1, dims=1).contiguous()
+    ks = torch.full((B, T), 64.0)
+    vs = torch.full((B, T), 32.0)
+    q = torch.randn(B, Hq, d, generator=g).bfloat16()
+    lengths = torch.tensor([T], dtype=torch.int32)
+    o, lse, idx = cuda_lib.hs2_decode_select(cuda(q), cuda(kc), cuda(vc), cuda(lengths), W, k,
+                                             kv="e4m3", k_scale=cuda(ks), v_scale=cuda(vs))
+    ora = oracle.decode_select(q, kc, vc, lengths, W, k, kv="e4m3", k_scale=ks, v_scale=vs,
+                               probe=idx.cpu())
+    assert max_abs(o.float().cpu().numpy(), ora["o"]) <= TOL_E4M3
+    assert max_abs(lse.cpu().numpy(), ora["lse"]) <= TOL_LSE
+    check_selection(idx.cpu().numpy(), ora, np.array([T - 1]), W, k)
+
+
+def test_decode_needles_recovered(cuda_lib):
+    x = _decode_case("e4m3", 4, 65536, 16, 128, 128, 1024, seed=inputs.seed_for(4, 3))
+    _, _, idx = run_decode(cuda_lib, x)
+    for b in range(4):
+        assert set(x.needle_pos[b].tolist()) <= set(idx[b].tolist())

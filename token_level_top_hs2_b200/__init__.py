@@ -1,0 +1,222 @@
+"""B200 (sm_100a) library for HySparse2's token-level KV Reuse hot path.
+
+Python binding of the C ABI in include/hs2.h, argument marshalling only: every
+step of the computation runs in the CUDA kernels of libhs2.so.  PyTorch is used
+for device memory and streams.  Loading fails loudly when the library is
+missing; there is no CPU fallback.
+
+Entry points (same names as the C ABI):
+  hs2_full_attn_select  full-attention layer + window/top-k selection (prefill)
+  hs2_sparse_attn       sparse layer over the inherited selection (prefill)
+  hs2_decode_select     decode full layer + selection, split over the cache
+  hs2_decode_sparse     decode sparse layer over the inherited selection
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhs2.so")
+
+HS2_OK = 0
+HS2_ERR_INVALID_ARG = 1
+HS2_ERR_UNSUPPORTED = 2
+HS2_ERR_WORKSPACE = 3
+HS2_ERR_CUDA = 4
+HS2_ERR_DEVICE_DATA = 5
+HS2_KV_BF16 = 0
+HS2_KV_E4M3 = 1
+
+EXPORTED = [
+    "hs2_status_string", "hs2_version", "hs2_full_attn_select_workspace",
+    "hs2_full_attn_select", "hs2_sparse_attn", "hs2_decode_select_workspace",
+    "hs2_decode_select", "hs2_decode_sparse", "hs2_get_last_device_error",
+]
+
+
+class Hs2Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+class PrefillShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("L", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("d", ctypes.c_int), ("W", ctypes.c_int), ("k", ctypes.c_int),
+                ("scale", ctypes.c_float)]
+
+
+class DecodeShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Tmax", ctypes.c_int), ("Hq", ctypes.c_int),
+                ("d", ctypes.c_int), ("W", ctypes.c_int), ("k", ctypes.c_int),
+                ("scale", ctypes.c_float), ("kv", ctypes.c_int)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libhs2.so (built by token_level_top_hs2_b200/build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"hs2 CUDA library not built: {path} is missing "
+                           "(run python token_level_top_hs2_b200/build.py)")
+    L = ctypes.CDLL(path)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+    P, D = ctypes.POINTER(PrefillShape), ctypes.POINTER(DecodeShape)
+    L.hs2_status_string.argtypes = [i32]
+    L.hs2_status_string.restype = ctypes.c_char_p
+    L.hs2_version.argtypes = []
+    L.hs2_version.restype = i32
+    L.hs2_full_attn_select_workspace.argtypes = [P]
+    L.hs2_full_attn_select_workspace.restype = sz
+    L.hs2_full_attn_select.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.hs2_full_attn_select.restype = i32
+    L.hs2_sparse_attn.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp]
+    L.hs2_sparse_attn.restype = i32
+    L.hs2_decode_select_workspace.argtypes = [D]
+    L.hs2_decode_select_workspace.restype = sz
+    L.hs2_decode_select.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.hs2_decode_select.restype = i32
+    L.hs2_decode_sparse.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.hs2_decode_sparse.restype = i32
+    L.hs2_get_last_device_error.argtypes = [vp]
+    L.hs2_get_last_device_error.restype = i32
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return load().hs2_status_string(status).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != HS2_OK:
+        raise Hs2Error(status, what)
+
+
+def _kv_code(kv) -> int:
+    if kv in (HS2_KV_BF16, "bf16"):
+        return HS2_KV_BF16
+    if kv in (HS2_KV_E4M3, "e4m3"):
+        return HS2_KV_E4M3
+    raise ValueError(f"kv must be 'bf16' or 'e4m3', got {kv!r}")
+
+
+def _u8(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.uint8) if t.dtype == torch.float8_e4m3fn else t
+
+
+def prefill_shape(B, L, Hq, d, W, k, scale=None) -> PrefillShape:
+    return PrefillShape(B, L, Hq, d, W, k, 1.0 / math.sqrt(d) if scale is None else scale)
+
+
+def decode_shape(B, Tmax, Hq, d, W, k, kv="e4m3", scale=None) -> DecodeShape:
+    return DecodeShape(B, Tmax, Hq, d, W, k, 1.0 / math.sqrt(d) if scale is None else scale,
+                       _kv_code(kv))
+
+
+def hs2_full_attn_select_workspace(shape: PrefillShape) -> int:
+    return load().hs2_full_attn_select_workspace(ctypes.byref(shape))
+
+
+def hs2_full_attn_select(q, k, v, W: int, k_top: int, *, scale=None, o=None, lse=None, idx=None,
+                         workspace=None, want_lse: bool = True, stream=None):
+    """q [B,L,Hq,d] bf16, k/v [B,L,d] bf16 (CUDA).  Returns (o, lse or None, idx)."""
+    B, L, Hq, d = q.shape
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    dev = q.device
+    o = torch.empty_like(q) if o is None else o
+    if lse is None and want_lse:
+        lse = torch.empty(B, L, Hq, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, L, W + k_top, dtype=torch.int32, device=dev) if idx is None else idx
+    need = hs2_full_attn_select_workspace(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = load().hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                     _ptr(lse), _ptr(idx), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hs2_full_attn_select")
+    return o, lse, idx
+
+
+def hs2_sparse_attn(q, k, v, idx, *, kv="bf16", k_scale=None, v_scale=None, W=None, k_top=None,
+                    scale=None, o=None, stream=None):
+    """q [B,L,Hq,d] bf16; k/v [B,L,d] bf16 or e4m3 codes; idx [B,L,S]. Returns o."""
+    B, L, Hq, d = q.shape
+    S = idx.shape[-1]
+    if W is None:
+        W, k_top = 1, S - 1
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    o = torch.empty_like(q) if o is None else o
+    st = load().hs2_sparse_attn(ctypes.byref(shape), _ptr(q), _ptr(_u8(k)), _ptr(_u8(v)),
+                                _kv_code(kv), _ptr(k_scale), _ptr(v_scale), _ptr(idx), _ptr(o),
+                                _stream(stream))
+    _check(st, "hs2_sparse_attn")
+    return o
+
+
+def hs2_decode_select_workspace(shape: DecodeShape) -> int:
+    return load().hs2_decode_select_workspace(ctypes.byref(shape))
+
+
+def hs2_decode_select(q, k_cache, v_cache, lengths, W: int, k_top: int, *, kv="e4m3",
+                      k_scale=None, v_scale=None, scale=None, o=None, lse=None, idx=None,
+                      workspace=None, want_lse: bool = True, stream=None):
+    """q [B,Hq,d] bf16; caches [B,Tmax,d]; lengths [B] int32 (CUDA). Returns (o, lse, idx)."""
+    B, Hq, d = q.shape
+    Tmax = k_cache.shape[1]
+    shape = decode_shape(B, Tmax, Hq, d, W, k_top, kv, scale)
+    dev = q.device
+    o = torch.empty_like(q) if o is None else o
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, W + k_top, dtype=torch.int32, device=dev) if idx is None else idx
+    need = hs2_decode_select_workspace(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = load().hs2_decode_select(ctypes.byref(shape), _ptr(q), _ptr(_u8(k_cache)),
+                                  _ptr(_u8(v_cache)), _ptr(k_scale), _ptr(v_scale),
+                                  _ptr(lengths), _ptr(o), _ptr(lse), _ptr(idx), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hs2_decode_select")
+    return o, lse, idx
+
+
+def hs2_decode_sparse(q, k_cache, v_cache, lengths, idx, *, kv="e4m3", k_scale=None,
+                      v_scale=None, W=None, k_top=None, scale=None, o=None, stream=None):
+    """q [B,Hq,d] bf16; idx [B,S] int32. Returns o [B,Hq,d] bf16."""
+    B, Hq, d = q.shape
+    Tmax = k_cache.shape[1]
+    S = idx.shape[-1]
+    if W is None:
+        W, k_top = 1, S - 1
+    shape = decode_shape(B, Tmax, Hq, d, W, k_top, kv, scale)
+    o = torch.empty_like(q) if o is None else o
+    st = load().hs2_decode_sparse(ctypes.byref(shape), _ptr(q), _ptr(_u8(k_cache)),
+                                  _ptr(_u8(v_cache)), _ptr(k_scale), _ptr(v_scale),
+                                  _ptr(lengths), _ptr(idx), _ptr(o), _stream(stream))
+    _check(st, "hs2_decode_sparse")
+    return o
+
+
+def hs2_get_last_device_error(stream=None) -> int:
+    """Synchronise the stream and return the first pending device-side status."""
+    return load().hs2_get_last_device_error(_stream(stream))

@@ -1,0 +1,273 @@
+// Device helpers shared by the hs2 kernels (sm_100a).
+//
+// Fragment conventions for the warp-level m16n8k16 MMA (PTX ISA, "Matrix
+// fragments for mma.m16n8k16"): lane = 4*g + c (g = lane/4, c = lane%4).
+//   A (16x16): a0 (row g, k 2c..2c+1), a1 (row g+8, k 2c..), a2 (row g, k 2c+8..),
+//              a3 (row g+8, k 2c+8..)
+//   B (16x8):  b0 (k 2c..2c+1, col g), b1 (k 2c+8..2c+9, col g)
+//   C (16x8):  c0,c1 (row g, cols 2c, 2c+1), c2,c3 (row g+8, cols 2c, 2c+1)
+// A contraction is invariant under any permutation of k applied to A and B
+// alike, and output columns may be permuted if the store undoes it; the gather
+// kernels use both freedoms so that every lane loads whole 16-byte pieces of a
+// K or V row straight from global memory.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#define HS2_DEV __device__ __forceinline__
+
+namespace hs2 {
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Device-side data flags (reported by hs2_get_last_device_error).
+enum : unsigned {
+    FLAG_BAD_LENGTH = 1u,   // decode length outside [1, Tmax]
+    FLAG_Q_RANGE = 2u,      // |q| beyond the fp16 range on an e4m3 path
+    FLAG_BAD_INDEX = 4u,    // a selection index outside [0, t]
+    FLAG_SCALE_RANGE = 8u,  // a V scale beyond 65504 on an e4m3 path
+};
+
+HS2_DEV uint32_t lane_id() { return threadIdx.x & 31; }
+
+HS2_DEV float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+HS2_DEV void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+HS2_DEV void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <bool F16>
+HS2_DEV void mma(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (F16)
+        mma_f16(d, a, b0, b1);
+    else
+        mma_bf16(d, a, b0, b1);
+}
+
+HS2_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// Two e4m3 codes sitting in the HIGH bytes of the two 16-bit halves of t
+// (low bytes ignored) -> f16x2 whose values are exactly e4m3 * 2^-8.
+// e4m3 is s.eeee.mmm with bias 7; f16 is s.eeeee.mmmmmmmmmm with bias 15.
+// Moving the 7 magnitude bits down by one places eeee.mmm at exponent bits
+// 13..10 and mantissa bits 9..7: a normal code becomes 2^(e-15)(1+m/8) and a
+// subnormal one (e = 0) (m/8)2^-14, i.e. the e4m3 value times 2^-8 in both
+// cases; the sign bit stays in place.
+HS2_DEV uint32_t e4m3_hi_to_f16x2(uint32_t t) {
+    return (t & 0x80008000u) | ((t >> 1) & 0x3F803F80u);
+}
+
+// Four e4m3 codes (bytes 0..3 of w) -> two f16x2: (byte0, byte1), (byte2, byte3),
+// each value = e4m3 * 2^-8.
+HS2_DEV void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    lo = e4m3_hi_to_f16x2(prmt(w, 0u, 0x1404u));  // bytes [0, b0, 0, b1]
+    hi = e4m3_hi_to_f16x2(prmt(w, 0u, 0x3424u));  // bytes [0, b2, 0, b3]
+}
+
+HS2_DEV uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+HS2_DEV uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <bool F16>
+HS2_DEV uint32_t pack2(float lo, float hi) {
+    if constexpr (F16)
+        return pack_f16(lo, hi);
+    else
+        return pack_bf16(lo, hi);
+}
+
+HS2_DEV float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+HS2_DEV float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Loads that bypass L1 allocation for data read once.
+HS2_DEV uint4 ldg_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+HS2_DEV uint4 ldg_nc(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+HS2_DEV void cp_async16(void* smem, const void* gmem, bool valid = true) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
+    int n = valid ? 16 : 0;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(n));
+}
+HS2_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+HS2_DEV void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N));
+}
+
+HS2_DEV void ldsm_x4(uint32_t (&r)[4], const void* p) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(p);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(s));
+}
+HS2_DEV void ldsm_x4_t(uint32_t (&r)[4], const void* p) {
+    uint32_t s = (uint32_t)__cvta_generic_to_shared(p);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(s));
+}
+
+// Selection key: larger is better.  High word = the score's fp32 bits (scores
+// are >= 0, so the bit pattern orders like the value); low word = ~position,
+// so that among equal scores the lower position wins.  Keys are unique.
+HS2_DEV uint64_t make_key(float score, uint32_t pos) {
+    return ((uint64_t)__float_as_uint(score) << 32) | (uint64_t)(~pos);
+}
+HS2_DEV uint32_t key_pos(uint64_t key) { return ~(uint32_t)key; }
+
+// ---------------------------------------------------------------------------
+// Radix select over unique 64-bit keys: returns T such that exactly `kk` keys
+// of keys[0..n) are >= T (requires 0 < kk <= n).  Most-significant 8-bit digit
+// first; stops as soon as the keys sharing the selected prefix are all taken.
+//
+// Warp version: one warp, hist = 256 ints of shared memory owned by the warp.
+template <class Get>
+HS2_DEV uint64_t warp_radix_threshold(Get get, int n, int kk, int* hist) {
+    const int lane = lane_id();
+    uint64_t prefix = 0, mask = 0;
+    int need = kk;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            uint64_t key = get(i);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        }
+        __syncwarp();
+        // lane owns digits 8*lane .. 8*lane+7; suffix sums from the top digit down
+        int loc[8];
+        int tot = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; i--) {
+            loc[i] = hist[lane * 8 + i];
+            tot += loc[i];
+        }
+        // inclusive suffix scan over lanes (higher lanes = higher digits)
+        int suf = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            int v = __shfl_down_sync(0xffffffffu, suf, o);
+            if (lane + o < 32) suf += v;
+        }
+        int above = suf - tot;  // count of keys with digit > 8*lane+7
+        int sel_digit = -1, sel_above = 0, sel_cnt = 0;
+#pragma unroll
+        for (int i = 7; i >= 0; i--) {
+            if (sel_digit < 0 && above < need && above + loc[i] >= need) {
+                sel_digit = lane * 8 + i;
+                sel_above = above;
+                sel_cnt = loc[i];
+            }
+            above += loc[i];
+        }
+        unsigned who = __ballot_sync(0xffffffffu, sel_digit >= 0);
+        int src = __ffs(who) - 1;
+        sel_digit = __shfl_sync(0xffffffffu, sel_digit, src);
+        sel_above = __shfl_sync(0xffffffffu, sel_above, src);
+        sel_cnt = __shfl_sync(0xffffffffu, sel_cnt, src);
+        __syncwarp();
+        need -= sel_above;
+        prefix |= (uint64_t)sel_digit << shift;
+        mask |= (uint64_t)255 << shift;
+        if (sel_cnt == need) break;
+    }
+    return prefix;
+}
+
+// Block version (all threads of the block call it; blockDim.x multiple of 32,
+// >= 256).  hist = 256 ints + 4 ints of scratch in shared memory.
+template <class Get>
+HS2_DEV uint64_t block_radix_threshold(Get get, int n, int kk, int* hist) {
+    const int tid = threadIdx.x;
+    int* sel = hist + 256;  // [digit, above, count]
+    uint64_t prefix = 0, mask = 0;
+    int need = kk;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += blockDim.x) {
+            uint64_t key = get(i);
+            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            const int lane = tid;
+            int loc[8];
+            int tot = 0;
+#pragma unroll
+            for (int i = 7; i >= 0; i--) {
+                loc[i] = hist[lane * 8 + i];
+                tot += loc[i];
+            }
+            int suf = tot;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                int v = __shfl_down_sync(0xffffffffu, suf, o);
+                if (lane + o < 32) suf += v;
+            }
+            int above = suf - tot;
+#pragma unroll
+            for (int i = 7; i >= 0; i--) {
+                if (above < need && above + loc[i] >= need) {
+                    sel[0] = lane * 8 + i;
+                    sel[1] = above;
+                    sel[2] = loc[i];
+                }
+                above += loc[i];
+            }
+        }
+        __syncthreads();
+        int digit = sel[0], sab = sel[1], scnt = sel[2];
+        __syncthreads();
+        need -= sab;
+        prefix |= (uint64_t)digit << shift;
+        mask |= (uint64_t)255 << shift;
+        if (scnt == need) break;
+    }
+    return prefix;
+}
+
+}  // namespace hs2

@@ -1,0 +1,386 @@
+// C ABI of the hs2 library (declared in include/hs2.h): argument validation,
+// workspace layout and kernel launches.  All kernels live in the headers
+// included below; this file is the library's single translation unit.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdio.h>
+
+#include "../../include/hs2.h"
+#include "decode_kernels.cuh"
+#include "prefill_kernels.cuh"
+#include "sparse_kernels.cuh"
+
+using namespace hs2;
+
+namespace {
+
+// Device-side data flags (FLAG_* in common.cuh); one word per device.
+__device__ unsigned g_device_flags;
+
+constexpr int kMaxDevices = 64;
+unsigned* g_flag_ptr[kMaxDevices];
+
+unsigned* device_flags() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_flag_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_flags) != cudaSuccess) return nullptr;
+        g_flag_ptr[dev] = static_cast<unsigned*>(p);
+    }
+    return g_flag_ptr[dev];
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+hs2_status check_common(int Hq, int d, int W, int k, float scale) {
+    if (!(scale > 0.f) || !isfinite(scale) || W < 1 || k < 0) return HS2_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return HS2_ERR_UNSUPPORTED;
+    if (Hq != 4 && Hq != 8 && Hq != 16) return HS2_ERR_UNSUPPORTED;
+    if ((long long)W + k > 2048) return HS2_ERR_UNSUPPORTED;
+    return HS2_OK;
+}
+
+hs2_status check_prefill(const hs2_prefill_shape* s) {
+    if (!s) return HS2_ERR_INVALID_ARG;
+    if (s->B < 1 || s->L < 1 || s->B > 65535) return HS2_ERR_INVALID_ARG;
+    return check_common(s->Hq, s->d, s->W, s->k, s->scale);
+}
+
+hs2_status check_decode(const hs2_decode_shape* s) {
+    if (!s) return HS2_ERR_INVALID_ARG;
+    if (s->B < 1 || s->Tmax < 1 || s->B > 65535) return HS2_ERR_INVALID_ARG;
+    if (s->kv != HS2_KV_BF16 && s->kv != HS2_KV_E4M3) return HS2_ERR_INVALID_ARG;
+    return check_common(s->Hq, s->d, s->W, s->k, s->scale);
+}
+
+hs2_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+template <class K>
+bool set_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return true;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)bytes) == cudaSuccess;
+}
+
+// ---------------------------------------------------------------- prefill
+int pf_cap(int k) { return (int)round_up((size_t)2 * k + 256, 32); }
+
+struct PrefillWs {
+    size_t lse_off, buf_off, total;
+};
+PrefillWs prefill_ws(const hs2_prefill_shape* s) {
+    PrefillWs w;
+    const size_t rows = (size_t)s->B * s->L;
+    w.lse_off = 0;
+    w.buf_off = round_up(rows * s->Hq * sizeof(float), 256);
+    w.total = w.buf_off + (s->k > 0 ? rows * pf_cap(s->k) * sizeof(uint64_t) : 0);
+    return w;
+}
+
+template <int D>
+hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void* k,
+                           const void* v, void* o, float* lse, int32_t* idx, uint8_t* ws,
+                           cudaStream_t st) {
+    const PrefillWs w = prefill_ws(s);
+    float* lse_p = lse ? lse : reinterpret_cast<float*>(ws + w.lse_off);
+    const float scale2 = s->scale * kLog2e;
+    {
+        const size_t smem = 4 * PF_BN * D * 2;
+        auto kern = prefill_pass1_kernel<D>;
+        if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+        dim3 grid((s->L + PF_BM - 1) / PF_BM, s->Hq / 2, s->B);
+        kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                      static_cast<const __nv_bfloat16*>(k),
+                                      static_cast<const __nv_bfloat16*>(v),
+                                      static_cast<__nv_bfloat16*>(o), lse_p, s->L, s->Hq, scale2);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    {
+        const size_t smem = 2 * PF_BN * D * 2 + (8 * PS_BM * PF_BN + PS_BM * PF_BN) * 4 +
+                            8 * 256 * 4 + PS_BM * sizeof(RowState);
+        auto kern = prefill_pass2_kernel<D>;
+        if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+        dim3 grid((s->L + PS_BM - 1) / PS_BM, s->B);
+        kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q),
+                                      static_cast<const __nv_bfloat16*>(k), lse_p, s->L, s->Hq,
+                                      s->W, s->k, s->W + s->k, pf_cap(s->k), scale2,
+                                      reinterpret_cast<uint64_t*>(ws + w.buf_off), idx);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    return HS2_OK;
+}
+
+template <int D, bool FP8>
+hs2_status run_sparse(const hs2_prefill_shape* s, const void* q, const void* k, const void* v,
+                      const float* ks, const float* vs, const int32_t* idx, void* o,
+                      cudaStream_t st, unsigned* flags) {
+    constexpr int WARPS = 4;
+    const int64_t n_tok = (int64_t)s->B * s->L;
+    const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
+    const int64_t blocks = (n_tok + WARPS - 1) / WARPS;
+    if (blocks > 0x7fffffff) return HS2_ERR_UNSUPPORTED;
+    sparse_prefill_kernel<D, FP8, WARPS><<<(unsigned)blocks, WARPS * 32, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const uint8_t*>(k),
+        static_cast<const uint8_t*>(v), ks, vs, idx, static_cast<__nv_bfloat16*>(o), n_tok, s->L,
+        s->Hq, s->W + s->k, qk_scale, flags);
+    return launch_status();
+}
+
+// ----------------------------------------------------------------- decode
+constexpr int kDecCh1 = 4096;   // pass-1 rows per CTA
+constexpr int kDecCh2 = 8192;   // pass-2 rows per CTA
+constexpr int kDecGroup = 8;    // chunk winners merged per CTA
+constexpr int kDecWarps = 8;
+
+struct DecodeWs {
+    int n1, n2, ng;
+    size_t cnt_off, lse2_off, part_off, cand_off, ccnt_off, gcand_off, gcnt_off, total;
+};
+DecodeWs decode_ws(const hs2_decode_shape* s) {
+    DecodeWs w;
+    const size_t B = s->B;
+    const int kk = s->k > 0 ? s->k : 1;
+    w.n1 = (s->Tmax + kDecCh1 - 1) / kDecCh1;
+    w.n2 = (s->Tmax + kDecCh2 - 1) / kDecCh2;
+    w.ng = (w.n2 + kDecGroup - 1) / kDecGroup;
+    const size_t part_floats = (size_t)16 * s->d + 32;
+    size_t off = 0;
+    w.cnt_off = off;  off = round_up(off + 2 * B * sizeof(unsigned), 256);
+    w.lse2_off = off; off = round_up(off + B * 16 * sizeof(float), 256);
+    w.part_off = off; off = round_up(off + B * w.n1 * part_floats * sizeof(float), 256);
+    w.cand_off = off; off = round_up(off + B * w.n2 * kk * sizeof(uint64_t), 256);
+    w.ccnt_off = off; off = round_up(off + B * w.n2 * sizeof(int), 256);
+    w.gcand_off = off; off = round_up(off + B * w.ng * kk * sizeof(uint64_t), 256);
+    w.gcnt_off = off; off = round_up(off + B * w.ng * sizeof(int), 256);
+    w.total = off;
+    return w;
+}
+
+template <int D, bool FP8>
+hs2_status run_decode_select(const hs2_decode_shape* s, const void* q, const void* kc,
+                             const void* vc, const float* ks, const float* vs,
+                             const int32_t* lengths, void* o, float* lse, int32_t* idx,
+                             uint8_t* ws, cudaStream_t st, unsigned* flags) {
+    const DecodeWs w = decode_ws(s);
+    unsigned* counters = reinterpret_cast<unsigned*>(ws + w.cnt_off);
+    float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
+    float* part = reinterpret_cast<float*>(ws + w.part_off);
+    uint64_t* cand = reinterpret_cast<uint64_t*>(ws + w.cand_off);
+    int* ccnt = reinterpret_cast<int*>(ws + w.ccnt_off);
+    uint64_t* gcand = reinterpret_cast<uint64_t*>(ws + w.gcand_off);
+    int* gcnt = reinterpret_cast<int*>(ws + w.gcnt_off);
+    const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
+    const auto* qp = static_cast<const __nv_bfloat16*>(q);
+    const auto* kp = static_cast<const uint8_t*>(kc);
+    const auto* vp = static_cast<const uint8_t*>(vc);
+
+    if (cudaMemsetAsync(counters, 0, 2 * (size_t)s->B * sizeof(unsigned), st) != cudaSuccess)
+        return HS2_ERR_CUDA;
+    {
+        const size_t smem = (size_t)kDecWarps * DecodePart<D>::FLOATS * sizeof(float);
+        auto kern = decode_pass1_kernel<D, FP8, kDecWarps>;
+        if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+        kern<<<dim3(w.n1, s->B), kDecWarps * 32, smem, st>>>(
+            qp, kp, vp, ks, vs, lengths, s->Tmax, s->Hq, kDecCh1, w.n1, qk_scale, part, counters,
+            lse2, lse, static_cast<__nv_bfloat16*>(o), flags);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    int n2 = w.n2, ng = w.ng;
+    if (s->k > 0) {
+        const size_t smem = (size_t)kDecCh2 * sizeof(float);
+        auto kern = decode_pass2_kernel<D, FP8, kDecWarps>;
+        if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+        kern<<<dim3(n2, s->B), kDecWarps * 32, smem, st>>>(qp, kp, ks, lengths, s->Tmax, s->Hq,
+                                                           s->W, s->k, kDecCh2, n2, qk_scale,
+                                                           lse2, cand, ccnt);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    } else {
+        n2 = 0;
+        ng = 1;
+    }
+    {
+        const int kk = s->k > 0 ? s->k : 1;
+        const size_t smem = ((size_t)kDecGroup * kk + kk) * sizeof(uint64_t);
+        if (!set_smem(decode_merge_kernel, smem)) return HS2_ERR_CUDA;
+        decode_merge_kernel<<<dim3(ng, s->B), 256, smem, st>>>(
+            cand, ccnt, n2, kDecGroup, ng, s->k, s->W, s->W + s->k, lengths, s->Tmax, gcand, gcnt,
+            counters + s->B, idx);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    return HS2_OK;
+}
+
+template <int D, bool FP8>
+hs2_status run_decode_sparse(const hs2_decode_shape* s, const void* q, const void* kc,
+                             const void* vc, const float* ks, const float* vs,
+                             const int32_t* lengths, const int32_t* idx, void* o,
+                             cudaStream_t st, unsigned* flags) {
+    constexpr int WARPS = 4, CLUSTER = 8;
+    const size_t smem = (size_t)(WARPS + 1) * (16 * D + 32) * sizeof(float);
+    auto kern = decode_sparse_kernel<D, FP8, WARPS, CLUSTER>;
+    if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(s->B * CLUSTER);
+    cfg.blockDim = dim3(WARPS * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CLUSTER;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(q),
+                                       static_cast<const uint8_t*>(kc),
+                                       static_cast<const uint8_t*>(vc), ks, vs, lengths, idx,
+                                       static_cast<__nv_bfloat16*>(o), s->Tmax, s->Hq,
+                                       s->W + s->k, qk_scale, flags);
+    return e == cudaSuccess ? launch_status() : HS2_ERR_CUDA;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* hs2_status_string(hs2_status s) {
+    switch (s) {
+        case HS2_OK: return "ok";
+        case HS2_ERR_INVALID_ARG: return "invalid argument";
+        case HS2_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case HS2_ERR_WORKSPACE: return "workspace too small";
+        case HS2_ERR_CUDA: return "CUDA error";
+        case HS2_ERR_DEVICE_DATA: return "out-of-contract data met on the device";
+    }
+    return "unknown status";
+}
+
+int hs2_version(void) { return 100; }
+
+size_t hs2_full_attn_select_workspace(const hs2_prefill_shape* shape) {
+    if (check_prefill(shape) != HS2_OK) return 0;
+    return prefill_ws(shape).total;
+}
+
+hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, const void* k,
+                                const void* v, void* o, float* lse, int32_t* idx,
+                                void* workspace, size_t workspace_bytes, hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !k || !v || !o || !idx || !workspace) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx) ||
+        !aligned16(workspace) || (lse && !aligned16(lse)))
+        return HS2_ERR_INVALID_ARG;
+    if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
+    if (workspace_bytes < prefill_ws(shape).total) return HS2_ERR_WORKSPACE;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (shape->d == 128) return run_full_select<128>(shape, q, k, v, o, lse, idx, ws, st);
+    return run_full_select<64>(shape, q, k, v, o, lse, idx, ws, st);
+}
+
+hs2_status hs2_sparse_attn(const hs2_prefill_shape* shape, const void* q, const void* k,
+                           const void* v, hs2_kv_dtype kv, const float* k_scale,
+                           const float* v_scale, const int32_t* idx, void* o,
+                           hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (kv != HS2_KV_BF16 && kv != HS2_KV_E4M3) return HS2_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !idx) return HS2_ERR_INVALID_ARG;
+    if (kv == HS2_KV_E4M3 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx))
+        return HS2_ERR_INVALID_ARG;
+    if (kv == HS2_KV_E4M3 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (kv == HS2_KV_E4M3)
+        return run_sparse<128, true>(shape, q, k, v, k_scale, v_scale, idx, o, st, flags);
+    if (shape->d == 128)
+        return run_sparse<128, false>(shape, q, k, v, nullptr, nullptr, idx, o, st, flags);
+    return run_sparse<64, false>(shape, q, k, v, nullptr, nullptr, idx, o, st, flags);
+}
+
+size_t hs2_decode_select_workspace(const hs2_decode_shape* shape) {
+    if (check_decode(shape) != HS2_OK) return 0;
+    return decode_ws(shape).total;
+}
+
+hs2_status hs2_decode_select(const hs2_decode_shape* shape, const void* q, const void* k_cache,
+                             const void* v_cache, const float* k_scale, const float* v_scale,
+                             const int32_t* lengths, void* o, float* lse, int32_t* idx,
+                             void* workspace, size_t workspace_bytes, hs2_stream_t stream) {
+    hs2_status e = check_decode(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !k_cache || !v_cache || !lengths || !o || !idx || !workspace)
+        return HS2_ERR_INVALID_ARG;
+    const bool fp8 = shape->kv == HS2_KV_E4M3;
+    if (fp8 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(idx) || !aligned16(workspace) || (lse && !aligned16(lse)))
+        return HS2_ERR_INVALID_ARG;
+    if (fp8 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
+    if (workspace_bytes < decode_ws(shape).total) return HS2_ERR_WORKSPACE;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (fp8)
+        return run_decode_select<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
+                                            o, lse, idx, ws, st, flags);
+    if (shape->d == 128)
+        return run_decode_select<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
+                                             lengths, o, lse, idx, ws, st, flags);
+    return run_decode_select<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths, o,
+                                        lse, idx, ws, st, flags);
+}
+
+hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const void* k_cache,
+                             const void* v_cache, const float* k_scale, const float* v_scale,
+                             const int32_t* lengths, const int32_t* idx, void* o,
+                             hs2_stream_t stream) {
+    hs2_status e = check_decode(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !k_cache || !v_cache || !lengths || !idx || !o) return HS2_ERR_INVALID_ARG;
+    const bool fp8 = shape->kv == HS2_KV_E4M3;
+    if (fp8 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(idx))
+        return HS2_ERR_INVALID_ARG;
+    if (fp8 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (fp8)
+        return run_decode_sparse<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
+                                            idx, o, st, flags);
+    if (shape->d == 128)
+        return run_decode_sparse<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
+                                             lengths, idx, o, st, flags);
+    return run_decode_sparse<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths,
+                                        idx, o, st, flags);
+}
+
+hs2_status hs2_get_last_device_error(hs2_stream_t stream) {
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HS2_ERR_CUDA;
+    if (cudaGetLastError() != cudaSuccess) return HS2_ERR_CUDA;
+    unsigned host = 0;
+    if (cudaMemcpyFromSymbol(&host, g_device_flags, sizeof host) != cudaSuccess)
+        return HS2_ERR_CUDA;
+    if (host) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_device_flags, &zero, sizeof zero) != cudaSuccess)
+            return HS2_ERR_CUDA;
+        return HS2_ERR_DEVICE_DATA;
+    }
+    return HS2_OK;
+}
+
+}  // extern "C"
