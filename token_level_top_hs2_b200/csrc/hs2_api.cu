@@ -59,11 +59,21 @@ hs2_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
+// Raise a kernel's dynamic shared-memory limit once per device (and per size
+// increase), so repeated calls -- including calls under stream capture -- make
+// no further attribute calls.
 template <class K>
 bool set_smem(K kernel, size_t bytes) {
     if (bytes <= 48 * 1024) return true;
-    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)bytes) == cudaSuccess;
+    static size_t done[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    if (done[dev] >= bytes) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+        cudaSuccess)
+        return false;
+    done[dev] = bytes;
+    return true;
 }
 
 // ---------------------------------------------------------------- prefill
