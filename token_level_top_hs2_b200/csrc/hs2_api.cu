@@ -5,6 +5,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "../../include/hs2.h"
 #include "decode_kernels.cuh"
 #include "prefill_kernels.cuh"
@@ -59,20 +61,39 @@ hs2_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
 
-// Raise a kernel's dynamic shared-memory limit once per device (and per size
-// increase), so repeated calls -- including calls under stream capture -- make
-// no further attribute calls.
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device) and
+// size increase, so repeated calls -- including calls under stream capture --
+// make no further attribute calls.
+struct SmemLimit {
+    const void* fn;
+    int dev;
+    size_t bytes;
+};
+SmemLimit g_smem_limits[512];
+int g_n_smem_limits = 0;
+std::mutex g_smem_mutex;
+
 template <class K>
 bool set_smem(K kernel, size_t bytes) {
     if (bytes <= 48 * 1024) return true;
-    static size_t done[kMaxDevices];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
-    if (done[dev] >= bytes) return true;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    const void* fn = reinterpret_cast<const void*>(kernel);
+    std::lock_guard<std::mutex> lock(g_smem_mutex);
+    SmemLimit* e = nullptr;
+    for (int i = 0; i < g_n_smem_limits; i++)
+        if (g_smem_limits[i].fn == fn && g_smem_limits[i].dev == dev) e = &g_smem_limits[i];
+    if (e && e->bytes >= bytes) return true;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
         cudaSuccess)
         return false;
-    done[dev] = bytes;
+    if (!e) {
+        if (g_n_smem_limits == 512) return true;  // table full: set again next time
+        e = &g_smem_limits[g_n_smem_limits++];
+        e->fn = fn;
+        e->dev = dev;
+    }
+    e->bytes = bytes;
     return true;
 }
 
