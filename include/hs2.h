@@ -163,6 +163,44 @@ hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const
                              const int32_t* lengths, const int32_t* idx, void* o,
                              hs2_stream_t stream);
 
+/* Size of the fixed device scratch used by hs2_decode_select_noalloc. */
+#define HS2_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * hs2_decode_select_noalloc: hs2_decode_select for callers that cannot
+ * allocate device memory.  The paper has no counterpart; this is a deployment
+ * convenience of this library.
+ *
+ * Some hosts own every byte of device memory: an inference server that
+ * reserves nearly all HBM for its KV-cache pool up front, a plugin whose host
+ * application exposes no allocator, or a latency-critical loop in which a
+ * cudaMalloc (which can synchronise the device) is not allowed.  Such callers
+ * cannot provide the workspace hs2_decode_select needs.  This entry point
+ * takes the same arguments minus the workspace and uses a fixed scratch area
+ * of HS2_NOALLOC_SCRATCH_BYTES that the library keeps in device memory
+ * (a file-scope __device__ array).  It allocates and frees nothing.
+ *
+ * Limits and behaviour:
+ *   - shapes whose hs2_decode_select_workspace() exceeds
+ *     HS2_NOALLOC_SCRATCH_BYTES are rejected with HS2_ERR_WORKSPACE before
+ *     anything is launched (B=16 x 256k and B=4 x 1M tokens fit);
+ *   - every GPU that loads the library holds the scratch until the process
+ *     exits;
+ *   - the first call on a device looks up the scratch address on that device
+ *     (it must be the current device); make that first call before any stream
+ *     capture;
+ *   - all calls on a device share the one scratch area and it keeps the last
+ *     call's contents (the parts that must start at zero are cleared by every
+ *     call), so calls whose execution overlaps on the GPU -- e.g. on two
+ *     streams without ordering -- race and give wrong results.  Serialise them.
+ * Results equal hs2_decode_select's for the same inputs.
+ */
+hs2_status hs2_decode_select_noalloc(const hs2_decode_shape* shape, const void* q,
+                                     const void* k_cache, const void* v_cache,
+                                     const float* k_scale, const float* v_scale,
+                                     const int32_t* lengths, void* o, float* lse, int32_t* idx,
+                                     hs2_stream_t stream);
+
 /*
  * Synchronises `stream`, then reports (and clears) the first error met since
  * the last call: a CUDA error (HS2_ERR_CUDA) or a device-side data flag

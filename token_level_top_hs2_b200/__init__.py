@@ -36,6 +36,7 @@ EXPORTED = [
     "hs2_status_string", "hs2_version", "hs2_full_attn_select_workspace",
     "hs2_full_attn_select", "hs2_sparse_attn", "hs2_decode_select_workspace",
     "hs2_decode_select", "hs2_decode_sparse", "hs2_get_last_device_error",
+    "hs2_decode_select_noalloc",
 ]
 
 
@@ -87,6 +88,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_decode_select.restype = i32
     L.hs2_decode_sparse.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.hs2_decode_sparse.restype = i32
+    L.hs2_decode_select_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.hs2_decode_select_noalloc.restype = i32
     L.hs2_get_last_device_error.argtypes = [vp]
     L.hs2_get_last_device_error.restype = i32
     _lib = L

@@ -415,3 +415,61 @@ hs2_status hs2_get_last_device_error(hs2_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ====================================================== no-allocation variant
+// hs2_decode_select_noalloc: decode select whose workspace is a fixed
+// file-scope device array instead of caller memory, for hosts that cannot
+// allocate device memory (see include/hs2.h).
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HS2_NOALLOC_SCRATCH_BYTES];
+
+uint8_t* g_noalloc_ptr[kMaxDevices];
+
+// Device address of the scratch on the current device, looked up once per
+// device.  In host code g_noalloc_scratch names a host-side stand-in, never
+// the device memory, so only this address may be handed to kernels.
+uint8_t* noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_noalloc_ptr[dev]) {
+        uint8_t* ptr = nullptr;
+        if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = ptr;
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" hs2_status hs2_decode_select_noalloc(const hs2_decode_shape* shape, const void* q,
+                                                const void* k_cache, const void* v_cache,
+                                                const float* k_scale, const float* v_scale,
+                                                const int32_t* lengths, void* o, float* lse,
+                                                int32_t* idx, hs2_stream_t stream) {
+    hs2_status e = check_decode(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !k_cache || !v_cache || !lengths || !o || !idx) return HS2_ERR_INVALID_ARG;
+    const bool fp8 = shape->kv == HS2_KV_E4M3;
+    if (fp8 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) ||
+        !aligned16(idx) || (lse && !aligned16(lse)))
+        return HS2_ERR_INVALID_ARG;
+    if (fp8 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
+    // the whole workspace layout of hs2_decode_select must fit the fixed scratch
+    if (decode_ws(shape).total > (size_t)HS2_NOALLOC_SCRATCH_BYTES) return HS2_ERR_WORKSPACE;
+    uint8_t* ws = noalloc_scratch();
+    if (!ws) return HS2_ERR_CUDA;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // run_decode_select clears the per-call counters at the start of every call
+    if (fp8)
+        return run_decode_select<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
+                                            o, lse, idx, ws, st, flags);
+    if (shape->d == 128)
+        return run_decode_select<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
+                                             lengths, o, lse, idx, ws, st, flags);
+    return run_decode_select<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths, o,
+                                        lse, idx, ws, st, flags);
+}
