@@ -60,7 +60,8 @@ typedef enum {
     HS2_ERR_UNSUPPORTED = 2,  /* valid but not implemented (d, Hq, W+k, dtype) */
     HS2_ERR_WORKSPACE = 3,    /* workspace smaller than the *_workspace() size */
     HS2_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
-    HS2_ERR_DEVICE_DATA = 5   /* a kernel met out-of-contract data (see above) */
+    HS2_ERR_DEVICE_DATA = 5,  /* a kernel met out-of-contract data (see above) */
+    HS2_ERR_TIMEOUT = 6       /* a bounded in-kernel wait gave up; results invalid */
 } hs2_status;
 
 typedef enum { HS2_KV_BF16 = 0, HS2_KV_E4M3 = 1 } hs2_kv_dtype;
@@ -203,8 +204,9 @@ hs2_status hs2_decode_select_noalloc(const hs2_decode_shape* shape, const void* 
 
 /*
  * Synchronises `stream`, then reports (and clears) the first error met since
- * the last call: a CUDA error (HS2_ERR_CUDA) or a device-side data flag
- * (HS2_ERR_DEVICE_DATA).  Returns HS2_OK when there is none.
+ * the last call: a CUDA error (HS2_ERR_CUDA), a pipeline wait inside a kernel
+ * that gave up after its time limit (HS2_ERR_TIMEOUT), or a device-side data
+ * flag (HS2_ERR_DEVICE_DATA).  Returns HS2_OK when there is none.
  */
 hs2_status hs2_get_last_device_error(hs2_stream_t stream);
 

@@ -41,7 +41,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(6):
+    for code in range(7):
         assert hs2.status_string(code) != "unknown status"
     assert hs2.status_string(99) == "unknown status"
     assert lib.hs2_version() >= 100

@@ -29,6 +29,7 @@ HS2_ERR_UNSUPPORTED = 2
 HS2_ERR_WORKSPACE = 3
 HS2_ERR_CUDA = 4
 HS2_ERR_DEVICE_DATA = 5
+HS2_ERR_TIMEOUT = 6
 HS2_KV_BF16 = 0
 HS2_KV_E4M3 = 1
 

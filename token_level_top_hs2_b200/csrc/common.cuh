@@ -29,6 +29,7 @@ enum : unsigned {
     FLAG_Q_RANGE = 2u,      // |q| beyond the fp16 range on an e4m3 path
     FLAG_BAD_INDEX = 4u,    // a selection index outside [0, t]
     FLAG_SCALE_RANGE = 8u,  // a V scale beyond 65504 on an e4m3 path
+    FLAG_TIMEOUT = 16u,     // a bounded wait inside a kernel gave up
 };
 
 HS2_DEV uint32_t lane_id() { return threadIdx.x & 31; }

@@ -1,7 +1,9 @@
 // C ABI of the hs2 library (declared in include/hs2.h): argument validation,
 // workspace layout and kernel launches.  All kernels live in the headers
 // included below; this file is the library's single translation unit.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 #include <math.h>
 #include <stdio.h>
 
@@ -10,6 +12,7 @@
 #include "../../include/hs2.h"
 #include "decode_kernels.cuh"
 #include "prefill_kernels.cuh"
+#include "prefill_tc.cuh"
 #include "sparse_kernels.cuh"
 
 using namespace hs2;
@@ -97,6 +100,51 @@ bool set_smem(K kernel, size_t bytes) {
     return true;
 }
 
+// ------------------------------------------------------------ tensor maps
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no direct
+// libcuda link).  bf16 tensors, 128-byte swizzle, 64-element inner box.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* p = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+bool map_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint32_t es[5] = {1, 1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides,
+               box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Q [B, L, Hq, D]: box of `rows` positions x 64 columns of one head.
+bool map_q(CUtensorMap* m, const void* q, int B, int L, int Hq, int D, int rows) {
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2,
+                                   (cuuint64_t)L * Hq * D * 2};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+    return map_bf16(m, q, 4, dims, strides, box);
+}
+
+// K or V [B, L, D]: box of `rows` positions x 64 columns.
+bool map_kv(CUtensorMap* m, const void* x, int B, int L, int D, int rows) {
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)L * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    return map_bf16(m, x, 3, dims, strides, box);
+}
+
 // ---------------------------------------------------------------- prefill
 int pf_cap(int k) { return (int)round_up((size_t)2 * k + 256, 32); }
 
@@ -115,19 +163,21 @@ PrefillWs prefill_ws(const hs2_prefill_shape* s) {
 template <int D>
 hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void* k,
                            const void* v, void* o, float* lse, int32_t* idx, uint8_t* ws,
-                           cudaStream_t st) {
+                           cudaStream_t st, unsigned* flags) {
     const PrefillWs w = prefill_ws(s);
     float* lse_p = lse ? lse : reinterpret_cast<float*>(ws + w.lse_off);
     const float scale2 = s->scale * kLog2e;
     {
-        const size_t smem = 4 * PF_BN * D * 2;
-        auto kern = prefill_pass1_kernel<D>;
+        CUtensorMap mq, mk, mv;
+        if (!map_q(&mq, q, s->B, s->L, s->Hq, D, tcfa::BM) ||
+            !map_kv(&mk, k, s->B, s->L, D, tcfa::BN) || !map_kv(&mv, v, s->B, s->L, D, tcfa::BN))
+            return HS2_ERR_CUDA;
+        const size_t smem = tcfa::Fwd<D>::SMEM;
+        auto kern = tcfa::prefill_fwd_tc_kernel<D>;
         if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
-        dim3 grid((s->L + PF_BM - 1) / PF_BM, s->Hq / 2, s->B);
-        kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                      static_cast<const __nv_bfloat16*>(k),
-                                      static_cast<const __nv_bfloat16*>(v),
-                                      static_cast<__nv_bfloat16*>(o), lse_p, s->L, s->Hq, scale2);
+        dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->Hq / 2, s->B);
+        kern<<<grid, 384, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse_p, s->L,
+                                      s->Hq, scale2, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     {
@@ -288,6 +338,7 @@ const char* hs2_status_string(hs2_status s) {
         case HS2_ERR_WORKSPACE: return "workspace too small";
         case HS2_ERR_CUDA: return "CUDA error";
         case HS2_ERR_DEVICE_DATA: return "out-of-contract data met on the device";
+        case HS2_ERR_TIMEOUT: return "a bounded wait inside a kernel timed out";
     }
     return "unknown status";
 }
@@ -310,10 +361,12 @@ hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, c
         return HS2_ERR_INVALID_ARG;
     if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
     if (workspace_bytes < prefill_ws(shape).total) return HS2_ERR_WORKSPACE;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    if (shape->d == 128) return run_full_select<128>(shape, q, k, v, o, lse, idx, ws, st);
-    return run_full_select<64>(shape, q, k, v, o, lse, idx, ws, st);
+    if (shape->d == 128) return run_full_select<128>(shape, q, k, v, o, lse, idx, ws, st, flags);
+    return run_full_select<64>(shape, q, k, v, o, lse, idx, ws, st, flags);
 }
 
 hs2_status hs2_sparse_attn(const hs2_prefill_shape* shape, const void* q, const void* k,
@@ -409,7 +462,7 @@ hs2_status hs2_get_last_device_error(hs2_stream_t stream) {
         const unsigned zero = 0;
         if (cudaMemcpyToSymbol(g_device_flags, &zero, sizeof zero) != cudaSuccess)
             return HS2_ERR_CUDA;
-        return HS2_ERR_DEVICE_DATA;
+        return (host & FLAG_TIMEOUT) ? HS2_ERR_TIMEOUT : HS2_ERR_DEVICE_DATA;
     }
     return HS2_OK;
 }
