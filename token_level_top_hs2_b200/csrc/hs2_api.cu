@@ -146,7 +146,8 @@ bool map_kv(CUtensorMap* m, const void* x, int B, int L, int D, int rows) {
 }
 
 // ---------------------------------------------------------------- prefill
-int pf_cap(int k) { return (int)round_up((size_t)2 * k + 256, 32); }
+// entries per (query row, key half) candidate stream
+int pf_cap(int k) { return (int)round_up((size_t)2 * k + 128, 32); }
 
 struct PrefillWs {
     size_t lse_off, buf_off, total;
@@ -156,7 +157,7 @@ PrefillWs prefill_ws(const hs2_prefill_shape* s) {
     const size_t rows = (size_t)s->B * s->L;
     w.lse_off = 0;
     w.buf_off = round_up(rows * s->Hq * sizeof(float), 256);
-    w.total = w.buf_off + (s->k > 0 ? rows * pf_cap(s->k) * sizeof(uint64_t) : 0);
+    w.total = w.buf_off + (s->k > 0 ? rows * 2 * pf_cap(s->k) * sizeof(uint64_t) : 0);
     return w;
 }
 
@@ -176,20 +177,22 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
         auto kern = tcfa::prefill_fwd_tc_kernel<D>;
         if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
         dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->Hq / 2, s->B);
-        kern<<<grid, 384, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse_p, s->L,
+        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse_p, s->L,
                                       s->Hq, scale2, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     {
-        const size_t smem = 2 * PF_BN * D * 2 + (8 * PS_BM * PF_BN + PS_BM * PF_BN) * 4 +
-                            8 * 256 * 4 + PS_BM * sizeof(RowState);
-        auto kern = prefill_pass2_kernel<D>;
+        CUtensorMap mq, mk;
+        if (!map_q(&mq, q, s->B, s->L, s->Hq, D, tcfa::BM) ||
+            !map_kv(&mk, k, s->B, s->L, D, tcfa::SBN))
+            return HS2_ERR_CUDA;
+        const size_t smem = tcfa::Sel<D>::SMEM;
+        auto kern = tcfa::prefill_select_tc_kernel<D>;
         if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
-        dim3 grid((s->L + PS_BM - 1) / PS_BM, s->B);
-        kern<<<grid, 256, smem, st>>>(static_cast<const __nv_bfloat16*>(q),
-                                      static_cast<const __nv_bfloat16*>(k), lse_p, s->L, s->Hq,
-                                      s->W, s->k, s->W + s->k, pf_cap(s->k), scale2,
-                                      reinterpret_cast<uint64_t*>(ws + w.buf_off), idx);
+        dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->B);
+        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
+                                      pf_cap(s->k), scale2,
+                                      reinterpret_cast<uint64_t*>(ws + w.buf_off), idx, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     return HS2_OK;

@@ -8,8 +8,10 @@
 //   warp 0        TMA producer (Q once, K/V through a 2-stage ring); TMEM owner
 //   warp 1        MMA issuer (one thread): S_h = Q_h K^T into TMEM, then
 //                 O_h += P_h V with P_h read from TMEM (it overwrites S_h)
-//   warps 4-7     softmax of head 0 (thread = query row = TMEM lane)
-//   warps 8-11    softmax of head 1
+//   warps 2-5     softmax of head 0 (thread = query row = TMEM lane; a warp
+//                 reaches TMEM lanes 32*(warp%4)..+31)
+//   warps 6-9     softmax of head 1
+// 320 threads leave 200 registers per thread for the 128-wide rows.
 // TMEM: S0 | S1 | O0 | O1.  The two heads are issued ping-pong so one head's
 // softmax overlaps the other head's GEMMs.  The running max is raised lazily
 // (only when a tile's max exceeds it by more than 2^8), so O is rescaled in
@@ -49,12 +51,11 @@ struct FwdBars {
     int abort_;
 };
 
-HS2_DEV void setmaxnreg_dec56() { asm volatile("setmaxnreg.dec.sync.aligned.u32 56;"); }
-HS2_DEV void setmaxnreg_inc224() { asm volatile("setmaxnreg.inc.sync.aligned.u32 224;"); }
+constexpr int kThreads = 320;  // 10 warps
 
-// grid (ceil(L/128), Hq/2, B), 384 threads.  Query blocks run longest first.
+// grid (ceil(L/128), Hq/2, B), 320 threads.  Query blocks run longest first.
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
@@ -99,8 +100,7 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     fence_after_sync();
     const uint32_t tmem = bars.tmem_base;
 
-    if (warp < 4) {
-        setmaxnreg_dec56();
+    if (warp < 2) {
         if (warp == 0 && lane == 0) {
             // ---------------------------------------------------- producer
             tma_prefetch_map(&map_q);
@@ -203,9 +203,8 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             mbar_wait(&bars.mma_drain, 0, &no_abort, flags);
         }
     } else {
-        setmaxnreg_inc224();
         // -------------------------------------------------------- softmax
-        const int hh = (warp >> 2) - 1;           // 0 for warps 4-7, 1 for 8-11
+        const int hh = (warp - 2) >> 2;           // 0 for warps 2-5, 1 for 6-9
         const int row = (warp & 3) * 32 + lane;    // query row in the block = TMEM lane
         const int t = qb * BM + row;
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
@@ -246,39 +245,32 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         break;
                     }
                     fence_after_sync();
-#pragma unroll
-                    for (int c = 0; c < D / 32; c++) {
-                        uint32_t r[32];
-                        tmem_ld32(o_col + c * 32, r);
+#pragma unroll 1
+                    for (int c = 0; c < D / 16; c++) {
+                        uint32_t r[16];
+                        tmem_ld16(o_col + c * 16, r);
                         tmem_ld_wait();
-                        uint32_t w0[16], w1[16];
 #pragma unroll
-                        for (int i = 0; i < 16; i++) {
-                            w0[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-                            w1[i] = __float_as_uint(__uint_as_float(r[16 + i]) * alpha);
-                        }
-                        tmem_st16(o_col + c * 32, w0);
-                        tmem_st16(o_col + c * 32 + 16, w1);
+                        for (int i = 0; i < 16; i++)
+                            r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+                        tmem_st16(o_col + c * 16, r);
                     }
                 }
                 m = mx;
             }
-            uint32_t pk[BN / 2];
             float rs = 0.f;
-#pragma unroll
-            for (int i = 0; i < BN / 2; i++) {
-                const float p0 = ex2(x[2 * i] - m), p1 = ex2(x[2 * i + 1] - m);
-                rs += p0 + p1;
-                pk[i] = pack_bf16(p0, p1);
-            }
-            l += rs;
 #pragma unroll
             for (int c = 0; c < BN / 32; c++) {
                 uint32_t w[16];
 #pragma unroll
-                for (int i = 0; i < 16; i++) w[i] = pk[c * 16 + i];
+                for (int i = 0; i < 16; i++) {
+                    const float p0 = ex2(x[c * 32 + 2 * i] - m), p1 = ex2(x[c * 32 + 2 * i + 1] - m);
+                    rs += p0 + p1;
+                    w[i] = pack_bf16(p0, p1);
+                }
                 tmem_st16(s_col + c * 16, w);
             }
+            l += rs;
             tmem_st_wait();
             fence_before_sync();
             __syncwarp();
@@ -309,6 +301,313 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
             }
             if (store) lse[((size_t)b * L + t) * Hq + h] = (m + __log2f(l)) * kLn2;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace tcfa
+}  // namespace hs2
+
+namespace hs2 {
+namespace tcfa {
+
+// Pass 2 (prefill_select_tc_kernel): head-summed probability scores and the
+// streaming per-row top-k, for one block of 128 query rows and ALL heads.
+// For every 256-key block and every head h the MMA warp computes
+// S = Q_h K^T (M=128, N=256) into one of two TMEM buffers; Q_h tiles stream
+// through a 2-stage TMA ring, the K block through another.  Score warps
+// (thread = query row; warps 2-5 own keys 0..127 of the block, warps 6-9 keys
+// 128..255) add 2^(S*scale*log2e - lse2_h) into 128 registers; after the last
+// head they hold score(t, s) for their 128 keys and feed the candidates
+// (s <= t-W) into the (row, half) stream: keys >= the stream's threshold are
+// appended to its workspace buffer; a buffer that would overflow is cut to its
+// k best by a warp radix select (one lane's buffer at a time), raising the
+// threshold.  At the end the two streams of a row are merged to exactly k.
+// The L x L score matrix never leaves the chip.
+constexpr int SBN = 256;   // keys per block
+constexpr int QSTAGE = 2;
+
+template <int D>
+struct Sel {
+    static constexpr int QT = BM * D * 2;     // Q tile of one head
+    static constexpr int KB = SBN * D * 2;    // K block
+    static constexpr int DB = D / 64;
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_Q = 2 * KB;
+    static constexpr int OFF_HIST = OFF_Q + QSTAGE * QT;         // 8 warps x 260 ints
+    static constexpr int OFF_CNT = OFF_HIST + 8 * 260 * 4;       // [2][128] ints
+    static constexpr int OFF_LSE = OFF_CNT + 2 * 128 * 4;        // [16][128] floats
+    static constexpr int SMEM = OFF_LSE + 16 * 128 * 4 + 1024;
+};
+
+struct SelBars {
+    uint64_t k_full[2], k_empty[2], q_full[QSTAGE], q_empty[QSTAGE];
+    uint64_t s_full[2], s_empty[2], mma_drain;
+    uint32_t tmem_base;
+    int abort_;
+};
+
+// Cut a stream buffer of `cnt` unique keys to its k best in place (one warp,
+// all lanes pass the same buf/cnt); returns the new threshold.
+HS2_DEV uint64_t warp_cut(uint64_t* buf, int cnt, int k, int* hist) {
+    const int lane = lane_id();
+    const uint64_t thr =
+        warp_radix_threshold([&](int i) { return __ldcg(buf + i); }, cnt, k, hist);
+    int wp = 0;
+    for (int i0 = 0; i0 < cnt; i0 += 32) {
+        const int i = i0 + lane;
+        const uint64_t key = i < cnt ? __ldcg(buf + i) : 0;
+        const bool keep = i < cnt && key >= thr;
+        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+        if (keep) __stcg(buf + wp + __popc(bal & ((1u << lane) - 1)), key);
+        wp += __popc(bal);
+    }
+    __syncwarp();
+    return thr;
+}
+
+// grid (ceil(L/128), B), 320 threads.  wsbuf: [B*L][2][cap] keys.
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
+                         const __grid_constant__ CUtensorMap map_k,
+                         const float* __restrict__ lse, int L, int Hq, int W, int kk, int S,
+                         int cap, float scale2, uint64_t* __restrict__ wsbuf,
+                         int32_t* __restrict__ idx, unsigned* __restrict__ flags) {
+    using F = Sel<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ SelBars bars;
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    const int nqb = (L + BM - 1) / BM;
+    const int qb = nqb - 1 - (int)blockIdx.x;
+    const int b = blockIdx.y;
+    const int last_key = (kk > 0) ? min(qb * BM + BM, L) - 1 - W : -1;  // candidates 0..last_key
+    const int n_kb = last_key >= 0 ? last_key / SBN + 1 : 0;
+    const int n_it = n_kb * Hq;
+    volatile int* abort_ = &bars.abort_;
+    int* cnts = reinterpret_cast<int*>(smem + F::OFF_CNT);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; i++) {
+            mbar_init(&bars.k_full[i], 1);
+            mbar_init(&bars.k_empty[i], 1);
+            mbar_init(&bars.s_full[i], 1);
+            mbar_init(&bars.s_empty[i], 8);
+        }
+        for (int i = 0; i < QSTAGE; i++) {
+            mbar_init(&bars.q_full[i], 1);
+            mbar_init(&bars.q_empty[i], 1);
+        }
+        mbar_init(&bars.mma_drain, 1);
+        bars.abort_ = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&bars.tmem_base, 512);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = bars.tmem_base;
+
+    if (warp < 2) {
+        if (warp == 0 && lane == 0 && n_it > 0) {
+            // ---------------------------------------------------- producer
+            tma_prefetch_map(&map_q);
+            tma_prefetch_map(&map_k);
+            int k_armed = 0, q_armed = 0;
+            for (int kb = 0; kb < n_kb && !*abort_; kb++) {
+                const int ks_ = kb & 1, ku = kb >> 1;
+                if (ku > 0 && !mbar_wait(&bars.k_empty[ks_], (ku - 1) & 1, abort_, flags)) break;
+                mbar_arrive_expect_tx(&bars.k_full[ks_], F::KB);
+                for (int db = 0; db < F::DB; db++)
+                    tma_load_3d(smem + F::OFF_K + ks_ * F::KB + db * (SBN * 128), &map_k, 64 * db,
+                                kb * SBN, b, &bars.k_full[ks_]);
+                k_armed++;
+                bool stop = false;
+                for (int h = 0; h < Hq; h++) {
+                    const int it = kb * Hq + h, qs = it % QSTAGE, qu = it / QSTAGE;
+                    if (qu > 0 && !mbar_wait(&bars.q_empty[qs], (qu - 1) & 1, abort_, flags)) {
+                        stop = true;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bars.q_full[qs], F::QT);
+                    for (int db = 0; db < F::DB; db++)
+                        tma_load_4d(smem + F::OFF_Q + qs * F::QT + db * (BM * 128), &map_q,
+                                    64 * db, h, qb * BM, b, &bars.q_full[qs]);
+                    q_armed++;
+                }
+                if (stop) break;
+            }
+            if (*abort_) {
+                volatile int no_abort = 0;
+                for (int j = max(0, k_armed - 2); j < k_armed; j++)
+                    mbar_wait(&bars.k_full[j & 1], (j >> 1) & 1, &no_abort, flags);
+                for (int j = max(0, q_armed - QSTAGE); j < q_armed; j++)
+                    mbar_wait(&bars.q_full[j % QSTAGE], (j / QSTAGE) & 1, &no_abort, flags);
+            }
+        } else if (warp == 1 && lane == 0 && n_it > 0) {
+            // ---------------------------------------------------- MMA issuer
+            constexpr uint32_t id = idesc_bf16_f32(BM, SBN, false, false);
+            for (int it = 0; it < n_it; it++) {
+                const int kb = it / Hq, h = it % Hq;
+                const int qs = it % QSTAGE, buf = it & 1;
+                if (h == 0 && !mbar_wait(&bars.k_full[kb & 1], (kb >> 1) & 1, abort_, flags))
+                    break;
+                if (!mbar_wait(&bars.q_full[qs], (it / QSTAGE) & 1, abort_, flags)) break;
+                if (it >= 2 && !mbar_wait(&bars.s_empty[buf], ((it >> 1) - 1) & 1, abort_, flags))
+                    break;
+                fence_after_sync();
+                const uint32_t a0 = smem_u32(smem + F::OFF_Q + qs * F::QT);
+                const uint32_t b0 = smem_u32(smem + F::OFF_K + (kb & 1) * F::KB);
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ks++) {
+                    const uint32_t ka = (ks >> 2) * (BM * 128) + (ks & 3) * 32;
+                    const uint32_t kbo = (ks >> 2) * (SBN * 128) + (ks & 3) * 32;
+                    mma_ss(tmem + buf * SBN, sdesc_sw128(a0 + ka, 16, 1024),
+                           sdesc_sw128(b0 + kbo, 16, 1024), id, ks > 0);
+                }
+                mma_commit(&bars.s_full[buf]);
+                mma_commit(&bars.q_empty[qs]);
+                if (h == Hq - 1) mma_commit(&bars.k_empty[kb & 1]);
+            }
+            mma_commit(&bars.mma_drain);
+            volatile int no_abort = 0;
+            mbar_wait(&bars.mma_drain, 0, &no_abort, flags);
+        }
+    } else {
+        // ---------------------------------------------------------- scores
+        const int half = (warp - 2) >> 2;        // keys half*128 .. +127 of each block
+        const int row = (warp & 3) * 32 + lane;  // TMEM lane
+        const int t = qb * BM + row;
+        const bool valid = t < L;
+        const int maxkey = t - W;                // candidates 0..maxkey
+        const uint32_t s_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 128;
+        int* hist = reinterpret_cast<int*>(smem + F::OFF_HIST) + (warp - 2) * 260;
+        uint64_t* my_buf = wsbuf + (((size_t)b * L + (valid ? t : 0)) * 2 + half) * cap;
+        // log2-domain lse of this row per head, in shared memory: [h][row]
+        float* lse2 = reinterpret_cast<float*>(smem + F::OFF_LSE);
+        if (half == 0)
+            for (int h = 0; h < 16; h++)
+                lse2[h * 128 + row] = (valid && h < Hq)
+                                          ? __ldg(lse + ((size_t)b * L + t) * Hq + h) * kLog2e
+                                          : INFINITY;
+        asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 score warps
+        int cnt = 0;
+        uint64_t thr = 0;
+        bool ok = true;
+        for (int kb = 0; kb < n_kb && ok; kb++) {
+            const int key0 = kb * SBN + half * 128;
+            const bool streams = valid && key0 <= maxkey;
+            {
+                // make room for this block's 128 candidates before accumulating
+                unsigned need = __ballot_sync(0xffffffffu, streams && cnt + 128 > cap);
+                while (need) {
+                    const int src = __ffs(need) - 1;
+                    need &= need - 1;
+                    uint64_t* sbuf = reinterpret_cast<uint64_t*>(
+                        __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(my_buf), src));
+                    const int scnt = __shfl_sync(0xffffffffu, cnt, src);
+                    const uint64_t nthr = warp_cut(sbuf, scnt, kk, hist);
+                    if (lane == src) {
+                        thr = nthr;
+                        cnt = kk;
+                    }
+                }
+            }
+            float acc[128];
+#pragma unroll
+            for (int i = 0; i < 128; i++) acc[i] = 0.f;
+            for (int h = 0; h < Hq; h++) {
+                const int it = kb * Hq + h, buf = it & 1;
+                if (!mbar_wait(&bars.s_full[buf], (it >> 1) & 1, abort_, flags)) {
+                    ok = false;
+                    break;
+                }
+                fence_after_sync();
+                const float l2 = lse2[h * 128 + row];
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    uint32_t r[16];
+                    tmem_ld16(s_lane + buf * SBN + c * 16, r);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; i++)
+                        acc[c * 16 + i] += ex2(fmaf(__uint_as_float(r[i]), scale2, -l2));
+                }
+                fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars.s_empty[buf]);
+            }
+            if (!ok) break;
+            // ---- all heads summed: stream the block's candidates
+            if (streams) {
+                // key >= thr on (score bits, ~position), compared as two words
+                const uint32_t thr_hi = (uint32_t)(thr >> 32), thr_lo = (uint32_t)thr;
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const int j = c * 16 + i;
+                        const uint32_t pos = (uint32_t)(key0 + j);
+                        const uint32_t sb = __float_as_uint(acc[j]);
+                        const bool take = (int)pos <= maxkey &&
+                                          (sb > thr_hi || (sb == thr_hi && ~pos >= thr_lo));
+                        if (take) {
+                            __stcg(my_buf + cnt, ((uint64_t)sb << 32) | (uint64_t)(~pos));
+                            cnt++;
+                        }
+                    }
+                    asm volatile("" ::: "memory");
+                }
+            }
+        }
+        cnts[half * 128 + row] = cnt;
+    }
+    fence_before_sync();
+    __syncthreads();
+    // ---------------------------------------------- final selection per row
+    // Warps 2..9: warp w takes rows w-2, w+6, ... (16 rows each); per row the
+    // union of its two streams is cut to exactly kk and written after the window.
+    if (warp >= 2 && !*abort_) {
+        int* hist = reinterpret_cast<int*>(smem + F::OFF_HIST) + (warp - 2) * 260;
+        for (int row = warp - 2; row < BM; row += 8) {
+            const int t = qb * BM + row;
+            if (t >= L) break;
+            const int n0 = cnts[row], n1 = cnts[128 + row];
+            const uint64_t* b0 = wsbuf + (((size_t)b * L + t) * 2 + 0) * cap;
+            const uint64_t* b1 = wsbuf + (((size_t)b * L + t) * 2 + 1) * cap;
+            auto get = [&](int i) { return i < n0 ? __ldcg(b0 + i) : __ldcg(b1 + (i - n0)); };
+            const int n = n0 + n1;
+            const int w0 = max(0, t - W + 1);
+            const int wl = t - w0 + 1;
+            int32_t* out = idx + ((size_t)b * L + t) * S;
+            for (int i = lane; i < wl; i += 32) out[i] = w0 + i;
+            int wp = wl;
+            if (n <= kk) {
+                for (int i = lane; i < n; i += 32) out[wl + i] = (int32_t)key_pos(get(i));
+                wp += n;
+            } else {
+                const uint64_t thr = warp_radix_threshold(get, n, kk, hist);
+                for (int i0 = 0; i0 < n; i0 += 32) {
+                    const int i = i0 + lane;
+                    const uint64_t key = i < n ? get(i) : 0;
+                    const bool keep = i < n && key >= thr;
+                    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                    if (keep) out[wp + __popc(bal & ((1u << lane) - 1))] = (int32_t)key_pos(key);
+                    wp += __popc(bal);
+                }
+            }
+            for (int i = wp + lane; i < S; i += 32) out[i] = -1;
         }
     }
     fence_before_sync();
