@@ -159,6 +159,49 @@ HS2_DEV uint64_t make_key(float score, uint32_t pos) {
 HS2_DEV uint32_t key_pos(uint64_t key) { return ~(uint32_t)key; }
 
 // ---------------------------------------------------------------------------
+// Suffix search over a 256-bin histogram held by one warp (hist[0..256)):
+// finds the highest bin j with sum_{i >= j} hist[i] >= need.  Returns j (or
+// -1 if the total is below need) and sets *above = sum_{i > j} hist[i],
+// *in_bin = hist[j].  Bins are read after a __syncwarp by the caller.
+HS2_DEV int warp_find_bin(const int* hist, int need, int* above_out, int* in_bin_out) {
+    const int lane = lane_id();
+    int loc[8];
+    int tot = 0;
+#pragma unroll
+    for (int i = 7; i >= 0; i--) {
+        loc[i] = hist[lane * 8 + i];
+        tot += loc[i];
+    }
+    int suf = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += v;
+    }
+    int above = suf - tot;
+    int sel = -1, sab = 0, scnt = 0;
+#pragma unroll
+    for (int i = 7; i >= 0; i--) {
+        if (sel < 0 && above < need && above + loc[i] >= need) {
+            sel = lane * 8 + i;
+            sab = above;
+            scnt = loc[i];
+        }
+        above += loc[i];
+    }
+    const unsigned who = __ballot_sync(0xffffffffu, sel >= 0);
+    if (!who) {
+        *above_out = 0;
+        *in_bin_out = 0;
+        return -1;
+    }
+    const int src = __ffs(who) - 1;
+    *above_out = __shfl_sync(0xffffffffu, sab, src);
+    *in_bin_out = __shfl_sync(0xffffffffu, scnt, src);
+    return __shfl_sync(0xffffffffu, sel, src);
+}
+
+// ---------------------------------------------------------------------------
 // Radix select over unique 64-bit keys: returns T such that exactly `kk` keys
 // of keys[0..n) are >= T (requires 0 < kk <= n).  Most-significant 8-bit digit
 // first; stops as soon as the keys sharing the selected prefix are all taken.

@@ -342,8 +342,12 @@ struct Sel {
     static constexpr int OFF_Q = 2 * KB;
     static constexpr int OFF_HIST = OFF_Q + QSTAGE * QT;         // 8 warps x 260 ints
     static constexpr int OFF_CNT = OFF_HIST + 8 * 260 * 4;       // [2][128] ints
-    static constexpr int OFF_LSE = OFF_CNT + 2 * 128 * 4;        // [16][128] floats
+    static constexpr int OFF_TB = OFF_CNT + 2 * 128 * 4;         // [2][128] threshold bits
+    static constexpr int OFF_LSE = OFF_TB + 2 * 128 * 4;         // [16][128] floats
     static constexpr int SMEM = OFF_LSE + 16 * 128 * 4 + 1024;
+    // final selection reuses the K region: per warp a boundary-bin buffer
+    static constexpr int BCAP = 1024;
+    static_assert(8 * BCAP * 8 <= 2 * KB, "boundary buffers must fit the K region");
 };
 
 struct SelBars {
@@ -352,6 +356,77 @@ struct SelBars {
     uint32_t tmem_base;
     int abort_;
 };
+
+// Score-bit histogram bins relative to a base: bin = (bits - base) >> 18, i.e.
+// 32 bins per octave over the 8 octaves above the base (higher scores clamp
+// into bin 255; scores below the base are not counted).
+constexpr int kBinShift = 18;
+HS2_DEV int rel_bin(uint32_t bits, uint32_t base) {
+    return bits < base ? -1 : (int)min((bits - base) >> kBinShift, 255u);
+}
+
+// Prune one candidate stream (warp-cooperative, all lanes pass the same
+// arguments): buf[0..cnt) holds unique keys, all with score bits >= tb, and
+// (once primed) at least k of them.  Two passes: a histogram of the score
+// bits relative to `base`, then keep every key in the highest bins that hold
+// >= k keys.  Returns the new count and sets *tb_out to the new threshold
+// bits (>= base); every key that can still reach the top k has score bits
+// >= it.  Returns -1 when no bin boundary frees room (the caller then falls
+// back to the exact cut).
+// Warp reads of a key list in batches of 8 per lane, so that the loads of a
+// batch are in flight together (the lists live in DRAM-backed workspace).
+constexpr int kBatch = 8;
+
+HS2_DEV int warp_prune(uint64_t* buf, int cnt, int k, int room, uint32_t base, int* hist,
+                       uint32_t* tb_out) {
+    const int lane = lane_id();
+#pragma unroll
+    for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
+    __syncwarp();
+    for (int i0 = 0; i0 < cnt; i0 += 32 * kBatch) {
+        uint64_t v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int i = i0 + u * 32 + lane;
+            v[u] = i < cnt ? __ldcg(buf + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int i = i0 + u * 32 + lane;
+            const int bn = i < cnt ? rel_bin((uint32_t)(v[u] >> 32), base) : -1;
+            if (bn >= 0) atomicAdd(&hist[bn], 1);
+        }
+    }
+    __syncwarp();
+    int above, in_bin;
+    const int j = warp_find_bin(hist, k, &above, &in_bin);
+    __syncwarp();
+    const int keep = above + in_bin;
+    if (j < 0 || keep > room) return -1;
+    const uint32_t tb = base + ((uint32_t)j << kBinShift);
+    // in-place compaction: a batch is fully read before any of its writes,
+    // and writes never pass the end of the batch
+    int wp = 0;
+    for (int i0 = 0; i0 < cnt; i0 += 32 * kBatch) {
+        uint64_t v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int i = i0 + u * 32 + lane;
+            v[u] = i < cnt ? __ldcg(buf + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int i = i0 + u * 32 + lane;
+            const bool kp = i < cnt && (uint32_t)(v[u] >> 32) >= tb;
+            const unsigned bal = __ballot_sync(0xffffffffu, kp);
+            if (kp) __stcg(buf + wp + __popc(bal & ((1u << lane) - 1)), v[u]);
+            wp += __popc(bal);
+        }
+    }
+    __syncwarp();
+    *tb_out = tb;
+    return wp;
+}
 
 // Cut a stream buffer of `cnt` unique keys to its k best in place (one warp,
 // all lanes pass the same buf/cnt); returns the new threshold.
@@ -394,6 +469,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     const int n_it = n_kb * Hq;
     volatile int* abort_ = &bars.abort_;
     int* cnts = reinterpret_cast<int*>(smem + F::OFF_CNT);
+    uint32_t* tbs = reinterpret_cast<uint32_t*>(smem + F::OFF_TB);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; i++) {
@@ -503,7 +579,10 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                                           : INFINITY;
         asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 score warps
         int cnt = 0;
-        uint64_t thr = 0;
+        uint32_t thr_bits = 0;  // appended keys have score bits >= thr_bits
+        // histogram origin of a stream's first prune: 1/64 of the row's mean
+        // score Hq/(t+1); later prunes start from the stream's threshold
+        const uint32_t base_bits = __float_as_uint((float)Hq / (64.f * (float)(t + 1)));
         bool ok = true;
         for (int kb = 0; kb < n_kb && ok; kb++) {
             const int key0 = kb * SBN + half * 128;
@@ -517,10 +596,17 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     uint64_t* sbuf = reinterpret_cast<uint64_t*>(
                         __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(my_buf), src));
                     const int scnt = __shfl_sync(0xffffffffu, cnt, src);
-                    const uint64_t nthr = warp_cut(sbuf, scnt, kk, hist);
+                    const uint32_t sbase = __shfl_sync(0xffffffffu, max(thr_bits, base_bits), src);
+                    uint32_t ntb = 0;
+                    int ncnt = warp_prune(sbuf, scnt, kk, cap - 128, sbase, hist, &ntb);
+                    if (ncnt < 0) {  // no histogram boundary frees room: exact cut to k
+                        const uint64_t nthr = warp_cut(sbuf, scnt, kk, hist);
+                        ntb = (uint32_t)(nthr >> 32);
+                        ncnt = kk;
+                    }
                     if (lane == src) {
-                        thr = nthr;
-                        cnt = kk;
+                        thr_bits = ntb;
+                        cnt = ncnt;
                     }
                 }
             }
@@ -551,8 +637,6 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             if (!ok) break;
             // ---- all heads summed: stream the block's candidates
             if (streams) {
-                // key >= thr on (score bits, ~position), compared as two words
-                const uint32_t thr_hi = (uint32_t)(thr >> 32), thr_lo = (uint32_t)thr;
 #pragma unroll
                 for (int c = 0; c < 8; c++) {
 #pragma unroll
@@ -560,8 +644,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         const int j = c * 16 + i;
                         const uint32_t pos = (uint32_t)(key0 + j);
                         const uint32_t sb = __float_as_uint(acc[j]);
-                        const bool take = (int)pos <= maxkey &&
-                                          (sb > thr_hi || (sb == thr_hi && ~pos >= thr_lo));
+                        const bool take = (int)pos <= maxkey && sb >= thr_bits;
                         if (take) {
                             __stcg(my_buf + cnt, ((uint64_t)sb << 32) | (uint64_t)(~pos));
                             cnt++;
@@ -572,14 +655,19 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             }
         }
         cnts[half * 128 + row] = cnt;
+        tbs[half * 128 + row] = thr_bits;
     }
     fence_before_sync();
     __syncthreads();
     // ---------------------------------------------- final selection per row
-    // Warps 2..9: warp w takes rows w-2, w+6, ... (16 rows each); per row the
-    // union of its two streams is cut to exactly kk and written after the window.
+    // Warps 2..9: warp w takes rows w-2, w+6, ... (16 rows each).  The union of
+    // a row's two streams is histogrammed relative to the higher stream
+    // threshold; keys above the boundary bin are written at once, the boundary
+    // bin is gathered into shared memory (the freed K region) and cut exactly
+    // there, so that exactly kk globals follow the window.
     if (warp >= 2 && !*abort_) {
         int* hist = reinterpret_cast<int*>(smem + F::OFF_HIST) + (warp - 2) * 260;
+        uint64_t* bnd = reinterpret_cast<uint64_t*>(smem + F::OFF_K) + (warp - 2) * F::BCAP;
         for (int row = warp - 2; row < BM; row += 8) {
             const int t = qb * BM + row;
             if (t >= L) break;
@@ -594,17 +682,91 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             for (int i = lane; i < wl; i += 32) out[i] = w0 + i;
             int wp = wl;
             if (n <= kk) {
-                for (int i = lane; i < n; i += 32) out[wl + i] = (int32_t)key_pos(get(i));
+                for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
+                    uint64_t v[kBatch];
+#pragma unroll
+                    for (int u = 0; u < kBatch; u++) {
+                        const int i = i0 + u * 32 + lane;
+                        v[u] = i < n ? get(i) : 0;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBatch; u++) {
+                        const int i = i0 + u * 32 + lane;
+                        if (i < n) out[wl + i] = (int32_t)key_pos(v[u]);
+                    }
+                }
                 wp += n;
             } else {
-                const uint64_t thr = warp_radix_threshold(get, n, kk, hist);
-                for (int i0 = 0; i0 < n; i0 += 32) {
-                    const int i = i0 + lane;
-                    const uint64_t key = i < n ? get(i) : 0;
-                    const bool keep = i < n && key >= thr;
-                    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-                    if (keep) out[wp + __popc(bal & ((1u << lane) - 1))] = (int32_t)key_pos(key);
-                    wp += __popc(bal);
+                const uint32_t base = max(tbs[row], tbs[128 + row]);
+#pragma unroll
+                for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
+                __syncwarp();
+                for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
+                    uint64_t v[kBatch];
+#pragma unroll
+                    for (int u = 0; u < kBatch; u++) {
+                        const int i = i0 + u * 32 + lane;
+                        v[u] = i < n ? get(i) : 0;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBatch; u++) {
+                        const int i = i0 + u * 32 + lane;
+                        const int bn = i < n ? rel_bin((uint32_t)(v[u] >> 32), base) : -1;
+                        if (bn >= 0) atomicAdd(&hist[bn], 1);
+                    }
+                }
+                __syncwarp();
+                int above, in_bin;
+                const int j = warp_find_bin(hist, kk, &above, &in_bin);
+                __syncwarp();
+                if (j >= 0 && in_bin <= F::BCAP) {
+                    // keys above bin j are in; bin j is gathered and cut exactly
+                    int nb = 0;
+                    for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
+                        uint64_t v[kBatch];
+#pragma unroll
+                        for (int u = 0; u < kBatch; u++) {
+                            const int i = i0 + u * 32 + lane;
+                            v[u] = i < n ? get(i) : 0;
+                        }
+#pragma unroll
+                        for (int u = 0; u < kBatch; u++) {
+                            const int i = i0 + u * 32 + lane;
+                            const uint64_t key = v[u];
+                            const int bn = i < n ? rel_bin((uint32_t)(key >> 32), base) : -1;
+                            const unsigned up = __ballot_sync(0xffffffffu, bn > j);
+                            const unsigned eq = __ballot_sync(0xffffffffu, bn == j);
+                            const unsigned lt = (1u << lane) - 1;
+                            if (bn > j) out[wp + __popc(up & lt)] = (int32_t)key_pos(key);
+                            if (bn == j) bnd[nb + __popc(eq & lt)] = key;
+                            wp += __popc(up);
+                            nb += __popc(eq);
+                        }
+                    }
+                    __syncwarp();
+                    const int need = kk - above;
+                    const uint64_t thr =
+                        warp_radix_threshold([&](int i) { return bnd[i]; }, nb, need, hist);
+                    for (int i0 = 0; i0 < nb; i0 += 32) {
+                        const int i = i0 + lane;
+                        const uint64_t key = i < nb ? bnd[i] : 0;
+                        const bool keep = i < nb && key >= thr;
+                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                        if (keep) out[wp + __popc(bal & ((1u << lane) - 1))] = (int32_t)key_pos(key);
+                        wp += __popc(bal);
+                    }
+                    __syncwarp();
+                } else {
+                    // fallback: exact radix select over the whole union
+                    const uint64_t thr = warp_radix_threshold(get, n, kk, hist);
+                    for (int i0 = 0; i0 < n; i0 += 32) {
+                        const int i = i0 + lane;
+                        const uint64_t key = i < n ? get(i) : 0;
+                        const bool keep = i < n && key >= thr;
+                        const unsigned bal = __ballot_sync(0xffffffffu, keep);
+                        if (keep) out[wp + __popc(bal & ((1u << lane) - 1))] = (int32_t)key_pos(key);
+                        wp += __popc(bal);
+                    }
                 }
             }
             for (int i = wp + lane; i < S; i += 32) out[i] = -1;
