@@ -37,7 +37,8 @@
  *     ascending first, then the global picks in no particular order, then -1
  *     padding.  |selection| = min(t+1, W+k).  Treat it as a set.
  *   - Device-side data checks (decode lengths outside [1, Tmax], a query value
- *     beyond the fp16 range +-65504 on an e4m3 path, an index outside [0, t])
+ *     beyond the fp16 range +-65504 or a V scale above 255 on an e4m3 path, an
+ *     index outside [0, t])
  *     do not fault: the kernel skips the offending work and records a flag that
  *     hs2_get_last_device_error reports as HS2_ERR_DEVICE_DATA.
  */
@@ -122,7 +123,7 @@ hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, c
  *   idx [B, L, S] int32, S = shape->W + shape->k: per token a set of positions
  *                               in [0, t], -1 entries ignored, no repeats
  *   o   [B, L, Hq, d] bf16      out; a token whose set is empty gets zeros
- * e4m3 additionally needs |q| <= 65504 and per-token scales <= 65504.
+ * e4m3 additionally needs |q| <= 65504 and per-token V scales <= 255.
  */
 hs2_status hs2_sparse_attn(const hs2_prefill_shape* shape, const void* q, const void* k,
                            const void* v, hs2_kv_dtype kv, const float* k_scale,
@@ -165,7 +166,7 @@ hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const
                              hs2_stream_t stream);
 
 /* Size of the fixed device scratch used by hs2_decode_select_noalloc. */
-#define HS2_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define HS2_NOALLOC_SCRATCH_BYTES (32u << 20)
 
 /*
  * hs2_decode_select_noalloc: hs2_decode_select for callers that cannot

@@ -166,6 +166,7 @@ def run_decode(hs2, x):
     ("e4m3", 2, 70000, 16, 128, 128, 1024, None),     # several merge groups
     ("bf16", 2, 5000, 8, 64, 32, 128, [5000, 77]),
     ("e4m3", 4, 300, 4, 128, 16, 0, [300, 1, 17, 250]),  # window only, length 1
+    ("e4m3", 2, 5001, 16, 128, 128, 256, [5001, 3000]),  # Tmax % 4 != 0: register path
 ])
 def test_decode_select_matches_oracle(cuda_lib, kv, B, T, Hq, d, W, k, lengths):
     x = _decode_case(kv, B, T, Hq, d, W, k, lengths, seed=inputs.seed_for(3, 7))

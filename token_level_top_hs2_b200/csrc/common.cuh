@@ -28,7 +28,7 @@ enum : unsigned {
     FLAG_BAD_LENGTH = 1u,   // decode length outside [1, Tmax]
     FLAG_Q_RANGE = 2u,      // |q| beyond the fp16 range on an e4m3 path
     FLAG_BAD_INDEX = 4u,    // a selection index outside [0, t]
-    FLAG_SCALE_RANGE = 8u,  // a V scale beyond 65504 on an e4m3 path
+    FLAG_SCALE_RANGE = 8u,  // a V scale beyond 255 on an e4m3 path
     FLAG_TIMEOUT = 16u,     // a bounded wait inside a kernel gave up
 };
 
@@ -86,6 +86,17 @@ HS2_DEV uint32_t e4m3_hi_to_f16x2(uint32_t t) {
 HS2_DEV void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
     lo = e4m3_hi_to_f16x2(prmt(w, 0u, 0x1404u));  // bytes [0, b0, 0, b1]
     hi = e4m3_hi_to_f16x2(prmt(w, 0u, 0x3424u));  // bytes [0, b2, 0, b3]
+}
+
+// Two e4m3 codes in the low 16 bits of w -> f16x2 of their exact values
+// (byte 0 -> low half).
+HS2_DEV uint32_t e4m3x2_lo_to_f16x2(uint32_t w) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %1;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+        : "=r"(r)
+        : "r"(w));
+    return r;
 }
 
 HS2_DEV uint32_t pack_bf16(float lo, float hi) {

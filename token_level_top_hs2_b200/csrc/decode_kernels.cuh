@@ -55,9 +55,9 @@ decode_pass1_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restri
     if (!wa.load_q(q + (size_t)b * Hq * D, Hq) && chunk == 0 && lane == 0 && warp == 0)
         atomicOr(flags, FLAG_Q_RANGE);
     if constexpr (FP8) {
-        // p*scale_v is held in f16: per-token V scales must stay within its range
+        // p*scale_v is held in f16 with p <= 2^8: per-token V scales must stay <= 255
         bool bad = false;
-        for (int s = s_begin + threadIdx.x; s < s_end; s += blockDim.x) bad |= !(vsb[s] <= 65504.f);
+        for (int s = s_begin + threadIdx.x; s < s_end; s += blockDim.x) bad |= !(vsb[s] <= 255.f);
         if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(flags, FLAG_SCALE_RANGE);
     }
     // tiles of 16 consecutive rows, interleaved over warps, one tile prefetched

@@ -13,9 +13,12 @@
 //   PV:   output n-tile jj, column g is element g*D/8 + jj; the lane reads the
 //         contiguous eighth [g*D/8, (g+1)*D/8) of the V rows of tile keys
 //         2c, 2c+1, 2c+8, 2c+9 and regroups them with byte permutes.
-// e4m3 rows become exact f16 values times 2^-8 (common.cuh) and the MMA runs
-// in f16 (Q is converted once; its |q| <= 65504 is checked); per-token scales
-// multiply the logit (K) and the probability (V) in fp32.
+// e4m3 K rows become exact f16 values times 2^-8 by a bit move (common.cuh),
+// e4m3 V rows exact f16 values by the hardware conversion, and the MMA runs
+// in f16 (Q is converted once; |q| <= 65504 is checked); per-token scales
+// multiply the logit (K) and the probability (V) in fp32.  Probabilities are
+// relative to a running max raised lazily, so they stay <= 2^8 and
+// p * v_scale fits f16 for v_scale <= 255.
 #pragma once
 
 #include "common.cuh"
@@ -41,6 +44,8 @@ struct TileRegs {
     float ks[4], vs[4];     // scales of tile keys 2c, 2c+1, 2c+8, 2c+9 (FP8)
     bool kval[4];           // validity of those four keys (lane's S columns)
 };
+
+constexpr float kLazyLog2 = 8.f;
 
 template <int D, bool FP8>
 struct WarpAttn {
@@ -165,26 +170,33 @@ struct WarpAttn {
             mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
             mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
         }
-        float alpha[2], mu[2];
+        // The running max is raised only when a tile's max exceeds it by more
+        // than 2^8 (log2 units); until then probabilities are taken relative
+        // to the older max and stay <= 2^8, and O/l need no rescale.
+        const bool up0 = mx[0] > m[0] + kLazyLog2, up1 = mx[1] > m[1] + kLazyLog2;
+        if (__any_sync(0xffffffffu, up0 || up1)) {
+            const float a0 = up0 ? ex2(m[0] - mx[0]) : 1.f;
+            const float a1 = up1 ? ex2(m[1] - mx[1]) : 1.f;
+            if (up0) m[0] = mx[0];
+            if (up1) m[1] = mx[1];
+            l[0] *= a0;
+            l[1] *= a1;
 #pragma unroll
-        for (int r = 0; r < 2; r++) {
-            float mn = fmaxf(m[r], mx[r]);
-            mu[r] = (mn == -INFINITY) ? 0.f : mn;
-            alpha[r] = ex2(m[r] - mu[r]);
-            m[r] = mn;
+            for (int jj = 0; jj < NT; jj++) {
+                o[jj][0] *= a0; o[jj][1] *= a0;
+                o[jj][2] *= a1; o[jj][3] *= a1;
+            }
         }
+        float mu[2];
+        mu[0] = (m[0] == -INFINITY) ? 0.f : m[0];
+        mu[1] = (m[1] == -INFINITY) ? 0.f : m[1];
         float p[2][4];
 #pragma unroll
         for (int j = 0; j < 2; j++)
 #pragma unroll
             for (int e = 0; e < 4; e++) p[j][e] = ex2(s[j][e] - mu[e >> 1]);
-        l[0] = l[0] * alpha[0] + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-        l[1] = l[1] * alpha[1] + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-#pragma unroll
-        for (int jj = 0; jj < NT; jj++) {
-            o[jj][0] *= alpha[0]; o[jj][1] *= alpha[0];
-            o[jj][2] *= alpha[1]; o[jj][3] *= alpha[1];
-        }
+        l[0] += (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+        l[1] += (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
         if constexpr (FP8) {
 #pragma unroll
             for (int j = 0; j < 2; j++)
@@ -200,14 +212,15 @@ struct WarpAttn {
         for (int jj = 0; jj < NT; jj++) {
             uint32_t b0, b1;
             if constexpr (FP8) {
+                // byte bi of two V rows -> the low 16 bits -> hardware e4m3x2 -> f16x2
                 const int wi = jj >> 2, bi = jj & 3;
-                const uint32_t sel = ((4u + bi) << 12) | ((4u + bi) << 8) | (bi << 4) | bi;
+                const uint32_t sel = ((4u + bi) << 4) | bi;
                 const uint32_t* v0 = reinterpret_cast<const uint32_t*>(&t.v[0][0]);
                 const uint32_t* v1 = reinterpret_cast<const uint32_t*>(&t.v[1][0]);
                 const uint32_t* v2 = reinterpret_cast<const uint32_t*>(&t.v[2][0]);
                 const uint32_t* v3 = reinterpret_cast<const uint32_t*>(&t.v[3][0]);
-                b0 = e4m3_hi_to_f16x2(prmt(v0[wi], v1[wi], sel));
-                b1 = e4m3_hi_to_f16x2(prmt(v2[wi], v3[wi], sel));
+                b0 = e4m3x2_lo_to_f16x2(prmt(v0[wi], v1[wi], sel));
+                b1 = e4m3x2_lo_to_f16x2(prmt(v2[wi], v3[wi], sel));
             } else {
                 const int wi = jj >> 1;
                 const uint32_t sel = (jj & 1) ? 0x7632u : 0x5410u;
@@ -231,8 +244,9 @@ struct WarpAttn {
         }
     }
 
-    // Output scale factor of the V codes (e4m3 values were held as value*2^-8).
-    static constexpr float kOutScale = FP8 ? 256.f : 1.f;
+    // Output scale of the accumulated V values (e4m3 V rows are converted
+    // exactly by the hardware conversion, so none is needed).
+    static constexpr float kOutScale = 1.f;
 
     // Store normalised O rows (< Hq) as bf16 into out [Hq, D].  Call finish_sums first.
     HS2_DEV void store(__nv_bfloat16* out, int Hq) const {

@@ -11,6 +11,7 @@
 
 #include "../../include/hs2.h"
 #include "decode_kernels.cuh"
+#include "decode_stream.cuh"
 #include "prefill_kernels.cuh"
 #include "prefill_tc.cuh"
 #include "sparse_kernels.cuh"
@@ -137,6 +138,34 @@ bool map_q(CUtensorMap* m, const void* q, int B, int L, int Hq, int D, int rows)
     return map_bf16(m, q, 4, dims, strides, box);
 }
 
+// Decode cache [B, Tmax, D] (e4m3 codes or bf16): box of 128 tokens x 128 bytes.
+bool map_cache(CUtensorMap* m, const void* x, int B, int Tmax, int D, bool fp8) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int esz = fp8 ? 1 : 2;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Tmax, (cuuint64_t)B};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * esz, (cuuint64_t)Tmax * D * esz};
+    const cuuint32_t box[3] = {(cuuint32_t)(128 / esz), (cuuint32_t)dec::TOK, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void*>(x), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Per-token scales [B, Tmax] fp32: box of 128 tokens (needs Tmax % 4 == 0).
+bool map_scales(CUtensorMap* m, const float* x, int B, int Tmax) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)Tmax, (cuuint64_t)B};
+    const cuuint64_t strides[1] = {(cuuint64_t)Tmax * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)dec::TOK, 1};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(x), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // K or V [B, L, D]: box of `rows` positions x 64 columns.
 bool map_kv(CUtensorMap* m, const void* x, int B, int L, int D, int rows) {
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)L, (cuuint64_t)B};
@@ -244,6 +273,109 @@ DecodeWs decode_ws(const hs2_decode_shape* s) {
     return w;
 }
 
+bool decode_streamable(const hs2_decode_shape* s);
+struct DecodeWs2;
+size_t decode_ws2_total(const hs2_decode_shape* s);
+size_t decode_ws_bytes(const hs2_decode_shape* s) {
+    return decode_streamable(s) ? decode_ws2_total(s) : decode_ws(s).total;
+}
+
+// TMA-fed decode path: usable unless e4m3 scales rows break TMA's 16-byte
+// stride rule (Tmax % 4 != 0 with more than one sequence).
+bool decode_streamable(const hs2_decode_shape* s) {
+    return !(s->kv == HS2_KV_E4M3 && (s->Tmax % 4) != 0 && s->B > 1);
+}
+
+struct DecodeWs2 {
+    int n_chunks, chunk_len, score_ld;
+    size_t zero_off, zero_bytes, lse2_off, part_off, score_off, bnd_off, total;
+};
+DecodeWs2 decode_ws2(const hs2_decode_shape* s) {
+    DecodeWs2 w;
+    const size_t B = s->B;
+    // at most one CTA per SM in total (a single wave), whole 128-token tiles per chunk
+    const int tiles = (s->Tmax + dec::TOK - 1) / dec::TOK;
+    int per_seq = 148 / s->B;
+    per_seq = per_seq < 1 ? 1 : (per_seq > tiles ? tiles : per_seq);
+    const int tiles_per_chunk = (tiles + per_seq - 1) / per_seq;
+    w.chunk_len = tiles_per_chunk * dec::TOK;
+    w.n_chunks = (s->Tmax + w.chunk_len - 1) / w.chunk_len;
+    const size_t part_floats = (size_t)16 * s->d + 32;
+    size_t off = 0;
+    // zeroed per call: pass-1 counter, gather counter, out count, boundary count, histogram
+    w.zero_off = off;
+    w.zero_bytes = B * (4 + 256) * sizeof(unsigned);
+    off = round_up(off + w.zero_bytes, 256);
+    w.lse2_off = off;  off = round_up(off + B * 16 * sizeof(float), 256);
+    w.part_off = off;  off = round_up(off + B * w.n_chunks * part_floats * sizeof(float), 256);
+    w.score_ld = (s->Tmax + 3) / 4 * 4;  // 16-byte rows
+    w.score_off = off; off = round_up(off + B * (size_t)w.score_ld * sizeof(float), 256);
+    w.bnd_off = off;   off = round_up(off + B * dec::BCAP * sizeof(uint64_t), 256);
+    w.total = off;
+    return w;
+}
+
+size_t decode_ws2_total(const hs2_decode_shape* s) { return decode_ws2(s).total; }
+
+template <int D, bool FP8>
+hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const void* kc,
+                             const void* vc, const float* ks, const float* vs,
+                             const int32_t* lengths, void* o, float* lse, int32_t* idx,
+                             uint8_t* ws, cudaStream_t st, unsigned* flags) {
+    using SG = dec::Stage<D, FP8>;
+    const DecodeWs2 w = decode_ws2(s);
+    const size_t B = s->B;
+    unsigned* zero = reinterpret_cast<unsigned*>(ws + w.zero_off);
+    unsigned* cnt1 = zero;
+    unsigned* cnt3 = zero + B;
+    unsigned* out_cnt = zero + 2 * B;
+    unsigned* bnd_cnt = zero + 3 * B;
+    unsigned* hist = zero + 4 * B;
+    float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
+    float* part = reinterpret_cast<float*>(ws + w.part_off);
+    float* scores = reinterpret_cast<float*>(ws + w.score_off);
+    uint64_t* bnd = reinterpret_cast<uint64_t*>(ws + w.bnd_off);
+    const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
+    CUtensorMap mk, mv, mks, mvs;
+    if (!map_cache(&mk, kc, s->B, s->Tmax, D, FP8) || !map_cache(&mv, vc, s->B, s->Tmax, D, FP8))
+        return HS2_ERR_CUDA;
+    if (FP8) {
+        if (!map_scales(&mks, ks, s->B, s->Tmax) || !map_scales(&mvs, vs, s->B, s->Tmax))
+            return HS2_ERR_CUDA;
+    } else {
+        mks = mk;  // unused placeholders
+        mvs = mk;
+    }
+    if (cudaMemsetAsync(zero, 0, w.zero_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
+    const auto* qp = static_cast<const __nv_bfloat16*>(q);
+    {
+        auto kern = dec::pass1_kernel<D, FP8>;
+        if (!set_smem(kern, SG::SMEM1)) return HS2_ERR_CUDA;
+        kern<<<dim3(w.n_chunks, s->B), dec::kThreads, SG::SMEM1, st>>>(
+            mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len, w.n_chunks, qk_scale, part,
+            cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), flags);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    if (s->k > 0) {
+        auto kern = dec::pass2_kernel<D, FP8>;
+        if (!set_smem(kern, SG::SMEM2)) return HS2_ERR_CUDA;
+        kern<<<dim3(w.n_chunks, s->B), dec::kThreads, SG::SMEM2, st>>>(
+            mk, mks, qp, lengths, s->Tmax, s->Hq, s->W, w.chunk_len, qk_scale, lse2, scores,
+            w.score_ld, hist, flags);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    {
+        const size_t smem = (size_t)dec::BCAP * sizeof(uint64_t);
+        if (!set_smem(dec::gather_kernel, smem)) return HS2_ERR_CUDA;
+        dec::gather_kernel<<<dim3(w.n_chunks, s->B), 256, smem, st>>>(
+            scores, w.score_ld, hist, lengths, s->Tmax, s->Hq, s->W, s->k, w.chunk_len, w.n_chunks,
+            out_cnt,
+            bnd_cnt, bnd, cnt3, idx);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+    }
+    return HS2_OK;
+}
+
 template <int D, bool FP8>
 hs2_status run_decode_select(const hs2_decode_shape* s, const void* q, const void* kc,
                              const void* vc, const float* ks, const float* vs,
@@ -296,6 +428,18 @@ hs2_status run_decode_select(const hs2_decode_shape* s, const void* q, const voi
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     return HS2_OK;
+}
+
+// Decode select: the TMA-fed streaming path, or the register path for the
+// shapes TMA cannot describe.
+template <int D, bool FP8>
+hs2_status run_decode(const hs2_decode_shape* s, const void* q, const void* kc, const void* vc,
+                      const float* ks, const float* vs, const int32_t* lengths, void* o,
+                      float* lse, int32_t* idx, uint8_t* ws, cudaStream_t st, unsigned* flags) {
+    if (decode_streamable(s))
+        return run_decode_stream<D, FP8>(s, q, kc, vc, ks, vs, lengths, o, lse, idx, ws, st,
+                                         flags);
+    return run_decode_select<D, FP8>(s, q, kc, vc, ks, vs, lengths, o, lse, idx, ws, st, flags);
 }
 
 template <int D, bool FP8>
@@ -396,7 +540,7 @@ hs2_status hs2_sparse_attn(const hs2_prefill_shape* shape, const void* q, const 
 
 size_t hs2_decode_select_workspace(const hs2_decode_shape* shape) {
     if (check_decode(shape) != HS2_OK) return 0;
-    return decode_ws(shape).total;
+    return decode_ws_bytes(shape);
 }
 
 hs2_status hs2_decode_select(const hs2_decode_shape* shape, const void* q, const void* k_cache,
@@ -413,18 +557,18 @@ hs2_status hs2_decode_select(const hs2_decode_shape* shape, const void* q, const
         !aligned16(idx) || !aligned16(workspace) || (lse && !aligned16(lse)))
         return HS2_ERR_INVALID_ARG;
     if (fp8 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
-    if (workspace_bytes < decode_ws(shape).total) return HS2_ERR_WORKSPACE;
+    if (workspace_bytes < decode_ws_bytes(shape)) return HS2_ERR_WORKSPACE;
     unsigned* flags = device_flags();
     if (!flags) return HS2_ERR_CUDA;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (fp8)
-        return run_decode_select<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
+        return run_decode<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
                                             o, lse, idx, ws, st, flags);
     if (shape->d == 128)
-        return run_decode_select<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
+        return run_decode<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
                                              lengths, o, lse, idx, ws, st, flags);
-    return run_decode_select<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths, o,
+    return run_decode<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths, o,
                                         lse, idx, ws, st, flags);
 }
 
@@ -513,7 +657,7 @@ extern "C" hs2_status hs2_decode_select_noalloc(const hs2_decode_shape* shape, c
         return HS2_ERR_INVALID_ARG;
     if (fp8 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
     // the whole workspace layout of hs2_decode_select must fit the fixed scratch
-    if (decode_ws(shape).total > (size_t)HS2_NOALLOC_SCRATCH_BYTES) return HS2_ERR_WORKSPACE;
+    if (decode_ws_bytes(shape) > (size_t)HS2_NOALLOC_SCRATCH_BYTES) return HS2_ERR_WORKSPACE;
     uint8_t* ws = noalloc_scratch();
     if (!ws) return HS2_ERR_CUDA;
     unsigned* flags = device_flags();
@@ -521,11 +665,11 @@ extern "C" hs2_status hs2_decode_select_noalloc(const hs2_decode_shape* shape, c
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     // run_decode_select clears the per-call counters at the start of every call
     if (fp8)
-        return run_decode_select<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
+        return run_decode<128, true>(shape, q, k_cache, v_cache, k_scale, v_scale, lengths,
                                             o, lse, idx, ws, st, flags);
     if (shape->d == 128)
-        return run_decode_select<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
+        return run_decode<128, false>(shape, q, k_cache, v_cache, nullptr, nullptr,
                                              lengths, o, lse, idx, ws, st, flags);
-    return run_decode_select<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths, o,
+    return run_decode<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths, o,
                                         lse, idx, ws, st, flags);
 }

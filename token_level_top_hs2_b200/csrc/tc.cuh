@@ -71,6 +71,13 @@ HS2_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsi
 // Tiled tensor loads (no multicast).  The tensor map lives in kernel
 // parameter space (__grid_constant__).  Coordinates are element indices,
 // innermost first.
+HS2_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 HS2_DEV void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
