@@ -12,6 +12,7 @@
 #include "../../include/hs2.h"
 #include "decode_kernels.cuh"
 #include "decode_stream.cuh"
+#include "decode_tc.cuh"
 #include "prefill_kernels.cuh"
 #include "prefill_tc.cuh"
 #include "sparse_kernels.cuh"
@@ -348,21 +349,38 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     }
     if (cudaMemsetAsync(zero, 0, w.zero_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
     const auto* qp = static_cast<const __nv_bfloat16*>(q);
-    {
+    if constexpr (FP8 && D == 128) {
+        // tensor-memory path: tokens as the MMA M dimension, exact f16 K/V
+        const float qk2 = s->scale * kLog2e;
+        using LY = dtc::Layout<true>;
+        using LY2 = dtc::Layout<false>;
+        if (!set_smem(dtc::pass1_tc_kernel, LY::SMEM)) return HS2_ERR_CUDA;
+        dtc::pass1_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kThreads, LY::SMEM, st>>>(
+            mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len, w.n_chunks, qk2, part,
+            cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), flags);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        if (s->k > 0) {
+            if (!set_smem(dtc::pass2_tc_kernel, LY2::SMEM)) return HS2_ERR_CUDA;
+            dtc::pass2_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kThreads, LY2::SMEM, st>>>(
+                mk, mks, qp, lengths, s->Tmax, s->Hq, s->W, w.chunk_len, qk2, lse2, scores,
+                w.score_ld, hist, flags);
+            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        }
+    } else {
         auto kern = dec::pass1_kernel<D, FP8>;
         if (!set_smem(kern, SG::SMEM1)) return HS2_ERR_CUDA;
         kern<<<dim3(w.n_chunks, s->B), dec::kThreads, SG::SMEM1, st>>>(
             mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len, w.n_chunks, qk_scale, part,
             cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-    }
-    if (s->k > 0) {
-        auto kern = dec::pass2_kernel<D, FP8>;
-        if (!set_smem(kern, SG::SMEM2)) return HS2_ERR_CUDA;
-        kern<<<dim3(w.n_chunks, s->B), dec::kThreads, SG::SMEM2, st>>>(
-            mk, mks, qp, lengths, s->Tmax, s->Hq, s->W, w.chunk_len, qk_scale, lse2, scores,
-            w.score_ld, hist, flags);
-        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        if (s->k > 0) {
+            auto kern2 = dec::pass2_kernel<D, FP8>;
+            if (!set_smem(kern2, SG::SMEM2)) return HS2_ERR_CUDA;
+            kern2<<<dim3(w.n_chunks, s->B), dec::kThreads, SG::SMEM2, st>>>(
+                mk, mks, qp, lengths, s->Tmax, s->Hq, s->W, w.chunk_len, qk_scale, lse2, scores,
+                w.score_ld, hist, flags);
+            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        }
     }
     {
         const size_t smem = (size_t)dec::BCAP * sizeof(uint64_t);
