@@ -166,7 +166,7 @@ hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const
                              hs2_stream_t stream);
 
 /* Size of the fixed device scratch used by hs2_decode_select_noalloc. */
-#define HS2_NOALLOC_SCRATCH_BYTES (32u << 20)
+#define HS2_NOALLOC_SCRATCH_BYTES (96u << 20)
 
 /*
  * hs2_decode_select_noalloc: hs2_decode_select for callers that cannot

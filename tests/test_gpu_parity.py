@@ -166,6 +166,7 @@ def run_decode(hs2, x):
     ("e4m3", 2, 70000, 16, 128, 128, 1024, None),     # several merge groups
     ("bf16", 2, 5000, 8, 64, 32, 128, [5000, 77]),
     ("e4m3", 4, 300, 4, 128, 16, 0, [300, 1, 17, 250]),  # window only, length 1
+    ("e4m3", 3, 9000, 4, 128, 64, 512, [9000, 4000, 600]),  # 4 heads, 12 padded
     ("e4m3", 2, 5001, 16, 128, 128, 256, [5001, 3000]),  # Tmax % 4 != 0: register path
 ])
 def test_decode_select_matches_oracle(cuda_lib, kv, B, T, Hq, d, W, k, lengths):
@@ -237,6 +238,30 @@ def test_e4m3_subnormal_codes_are_exact(cuda_lib):
     assert max_abs(o.float().cpu().numpy(), ora["o"]) <= TOL_E4M3
     assert max_abs(lse.cpu().numpy(), ora["lse"]) <= TOL_LSE
     check_selection(idx.cpu().numpy(), ora, np.array([T - 1]), W, k)
+
+
+def test_decode_select_exact_ties_take_lower_index(cuda_lib):
+    """Sequences whose older keys are all one row: every candidate score ties.
+
+    Sequence 0 has far more tied candidates than the sketch selection's
+    boundary buffer, so it goes through the exact fallback; sequence 2's tied
+    candidates fit, so the sketch path rescoring cuts them; sequence 1 is
+    ordinary.  Ties must go to the lower position in both paths."""
+    B, T, Hq, d, W, k = 3, 20000, 16, 128, 128, 1024
+    x = _decode_case("e4m3", B, T, Hq, d, W, k, [20000, 15000, 3000], seed=21)
+    for b in (0, 2):
+        x.k_cache[b, :] = x.k_cache[b, 5]
+        x.k_scale[b, :] = x.k_scale[b, 5]
+    o, lse, idx = run_decode(cuda_lib, x)
+    ora = oracle.decode_select(x.q, x.k_cache, x.v_cache, x.lengths, W, k, kv="e4m3",
+                               k_scale=x.k_scale, v_scale=x.v_scale, probe=idx)
+    assert max_abs(o, ora["o"]) <= TOL_E4M3
+    assert max_abs(lse, ora["lse"]) <= TOL_LSE
+    t = x.lengths.numpy().astype(np.int64) - 1
+    check_structure(idx, t, W, k)
+    check_selection(idx, ora, t, W, k)
+    for b in (0, 2):
+        assert sorted(idx[b, W:W + k].tolist()) == list(range(k))
 
 
 def test_decode_needles_recovered(cuda_lib):

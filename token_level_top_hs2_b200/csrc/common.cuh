@@ -70,6 +70,19 @@ HS2_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
+// Two floats -> f16x2 rounded toward zero: lo in bits 0..15, hi in bits 16..31.
+HS2_DEV uint32_t f16x2_rz(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rz.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// f16x2 bit pattern -> the two values as floats (exact).
+HS2_DEV float2 f16x2_to_float2(uint32_t h) {
+    __half2 v = *reinterpret_cast<__half2*>(&h);
+    return __half22float2(v);
+}
+
 // Two e4m3 codes sitting in the HIGH bytes of the two 16-bit halves of t
 // (low bytes ignored) -> f16x2 whose values are exactly e4m3 * 2^-8.
 // e4m3 is s.eeee.mmm with bias 7; f16 is s.eeeee.mmmmmmmmmm with bias 15.

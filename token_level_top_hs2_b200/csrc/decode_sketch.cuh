@@ -1,0 +1,283 @@
+// Decode selection from a per-token sketch (FP8 e4m3 cache, d = 128).
+//
+// HySparse2 summary (onedev.kr/papers/146), 'How it works': the full layer
+// ranks every older token by its exact attention score, here the sum over
+// query heads of the softmax probability,
+//     score(s) = sum_h 2^(x_h(s) - lse2_h),   x_h(s) = scale * log2(e) * <q_h, k_s>,
+// and keeps the top k (ties to the lower position) besides the window.
+//
+// lse2_h needs the whole cache, so a single streaming pass cannot form the
+// score.  Instead of reading K a second time, pass 1 leaves behind, for every
+// token, one byte per head: the top 8 bits (5 exponent and 3 mantissa bits)
+// of the f16 of p_h = 2^(x_h - R_h), rounded toward zero, where R_h is the
+// chunk's softmax reference for that 128-token tile (saved per tile).  A code
+// c therefore brackets p_h:  F(c) <= p_h < F(c + 1),  F(c) = the f16 with
+// bits c << 7.  For a normal F(c), F(c + 1) <= 9/8 F(c); codes below 2^-14
+// are subnormal and step by 2^-17.  With w_h = 2^(R_h - lse2_h) <= 2^-6
+// (R_h sits kSk = 6 below a running maximum, itself <= lse2_h),
+//     L(s) = sum_h w_h F(c_h)  <=  score(s)  <=  9/8 L(s) + Hq 2^-23.
+//
+// sketch_score_kernel   L(s) for every older token, and a 256-bin histogram
+//                       of L per sequence (1/16-octave bins);
+// sketch_gather_kernel  the bin holding the k-th largest L gives E, a lower
+//                       bound of the k-th largest score.  A token can be in
+//                       the top k only if 9/8 L + eps >= E; exactly those are
+//                       rescored from their K rows (a thread per token) and
+//                       the exact top k is cut from them.
+// If a sequence's candidates overflow the boundary buffer (many near-equal
+// scores, e.g. repeated keys), it is flagged and the exact pass 2 and its
+// gather run for that sequence instead (their launches are gated on the flag).
+#pragma once
+
+#include "decode_tc.cuh"
+
+namespace hs2 {
+namespace dsk {
+
+constexpr int TOK = 128;
+constexpr int kScoreThreads = 256;
+constexpr int kGatherThreads = 256;
+constexpr int kCandCap = 2048;  // candidates one CTA may rescore
+
+// ----------------------------------------------------------------------------
+// L(s) per token and the per-sequence histogram.  grid (G, B): the CTAs of a
+// sequence stride over its 128-token tiles, a warp per tile, two tiles of
+// codes in flight per warp.
+__global__ void __launch_bounds__(kScoreThreads)
+sketch_score_kernel(const uint8_t* __restrict__ sketch, const float* __restrict__ rsnap,
+                    int sk_tiles, const int32_t* __restrict__ lengths, int Tmax, int Hq, int W,
+                    int k, const float* __restrict__ lse2_ws, float* __restrict__ lrow,
+                    int score_ld, unsigned* __restrict__ hist_g) {
+    __shared__ unsigned hist[256];
+    const int b = blockIdx.y;
+    const int T = __ldg(lengths + b);
+    const int n_cand = (T >= 1 && T <= Tmax) ? max(0, T - W) : 0;
+    if (k <= 0 || n_cand <= k) return;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    constexpr int NW = kScoreThreads / 32;
+    const uint32_t base = dec::seq_base(Hq, T);
+    const float l2h = (lane & 15) < Hq ? __ldcg(lse2_ws + b * 16 + (lane & 15)) : INFINITY;
+    float* srow = lrow + (size_t)b * score_ld;
+    const uint8_t* sk_b = sketch + (size_t)b * Tmax * 16;
+    const float* rs_b = rsnap + (size_t)b * sk_tiles * 16;
+    const int n_tiles = (n_cand + TOK - 1) / TOK;
+    const int stride = gridDim.x * NW;
+    for (int g0 = blockIdx.x * NW + warp; g0 < n_tiles; g0 += 2 * stride) {
+        uint4 cw[2][4];
+        float rv[2];
+#pragma unroll
+        for (int v = 0; v < 2; v++) {
+            const int g = g0 + v * stride;
+            rv[v] = g < n_tiles ? __ldcg(rs_b + (size_t)g * 16 + (lane & 15)) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int tok = g * TOK + u * 32 + lane;
+                cw[v][u] = (g < n_tiles && tok < n_cand)
+                               ? __ldcg(reinterpret_cast<const uint4*>(sk_b + (size_t)tok * 16))
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < 2; v++) {
+            const int g = g0 + v * stride;
+            if (g >= n_tiles) break;
+            // tile weights w_h = 2^(R_h - lse2_h), zero for padded heads
+            const float wl = ((lane & 15) < Hq && rv[v] != -INFINITY) ? ex2(rv[v] - l2h) : 0.f;
+            float w[16];
+#pragma unroll
+            for (int h = 0; h < 16; h++) w[h] = __shfl_sync(0xffffffffu, wl, h);
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const int tok = g * TOK + u * 32 + lane;
+                const uint32_t wd[4] = {cw[v][u].x, cw[v][u].y, cw[v][u].z, cw[v][u].w};
+                float L = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    // codes of heads 4i..4i+3 -> f16 bit patterns c << 7
+                    const float2 a = f16x2_to_float2(prmt(wd[i], 0u, 0x1404u) >> 1);
+                    const float2 c = f16x2_to_float2(prmt(wd[i], 0u, 0x3424u) >> 1);
+                    L = fmaf(w[4 * i], a.x, L);
+                    L = fmaf(w[4 * i + 1], a.y, L);
+                    L = fmaf(w[4 * i + 2], c.x, L);
+                    L = fmaf(w[4 * i + 3], c.y, L);
+                }
+                const bool valid = tok < n_cand;
+                if (valid) srow[tok] = L;
+                const int bn = valid ? dec::score_bin(__float_as_uint(L), base) : -1;
+                const unsigned grp = __match_any_sync(0xffffffffu, bn);
+                if (valid && lane == __ffs(grp) - 1) atomicAdd(&hist[bn], (unsigned)__popc(grp));
+            }
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256; i += blockDim.x)
+        if (hist[i]) atomicAdd(hist_g + b * 256 + i, hist[i]);
+}
+
+struct GatherShared {
+    float q[16][128];     // f16-rounded query, as the MMA operand saw it
+    int cand[kCandCap];   // this CTA's candidate positions
+    int hist[260];
+    int bin;
+    unsigned n_cand, last;
+};
+
+// ----------------------------------------------------------------------------
+// Candidates, exact rescoring and the cut.  grid (n_chunks, B), 256 threads,
+// dynamic shared memory BCAP keys (used by the last CTA of each sequence).
+// A thread rescores one candidate at a time from its K row: the same
+// expression the exact pass evaluates, sum_h 2^(<q_h, k_s> sK qk2 - lse2_h).
+__global__ void __launch_bounds__(kGatherThreads)
+sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigned* __restrict__ hist_g,
+                     const uint8_t* __restrict__ kc, const float* __restrict__ ksc,
+                     const __nv_bfloat16* __restrict__ q, const float* __restrict__ lse2_ws,
+                     float qk2, const int32_t* __restrict__ lengths, int Tmax, int Hq, int W, int k,
+                     int chunk_len, int n_chunks, unsigned* __restrict__ bnd_cnt,
+                     uint64_t* __restrict__ bnd, unsigned* __restrict__ ovf,
+                     unsigned* __restrict__ counter, unsigned* __restrict__ out_cnt,
+                     int32_t* __restrict__ idx) {
+    extern __shared__ uint64_t skeys[];
+    __shared__ GatherShared sh;
+    const int b = blockIdx.y, chunk = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    const int T = __ldg(lengths + b);
+    const bool ok = T >= 1 && T <= Tmax;
+    const int n_cand = ok ? max(0, T - W) : 0;
+    const int t = T - 1;
+    const int wl = ok ? min(T, W) : 0;
+    const int S = W + k;
+    int32_t* row = idx + (size_t)b * S;
+    const int s_begin = chunk * chunk_len;
+    const int s_end = min(s_begin + chunk_len, n_cand);
+    const bool ranked = k > 0 && n_cand > k;
+    if (ranked && s_end > s_begin) {
+        if (warp == 0) {
+            for (int i = lane; i < 256; i += 32) sh.hist[i] = (int)__ldcg(hist_g + b * 256 + i);
+            __syncwarp();
+            int above, in_bin;
+            const int j = warp_find_bin(sh.hist, k, &above, &in_bin);
+            if (lane == 0) {
+                sh.bin = j;
+                sh.n_cand = 0;
+            }
+        }
+        const __nv_bfloat16* qb = q + (size_t)b * Hq * 128;
+        for (int e = threadIdx.x; e < 16 * 128; e += blockDim.x) {
+            const int h = e >> 7;
+            sh.q[h][e & 127] =
+                h < Hq ? __half2float(__float2half_rn(__bfloat162float(qb[e]))) : 0.f;
+        }
+        __syncthreads();
+        const int j = sh.bin;
+        const uint32_t base = dec::seq_base(Hq, T);
+        // E <= the k-th largest L <= the k-th largest score; a token with
+        // 9/8 L + eps < E is out.  The factor (1 - 2^-10) absorbs rounding in
+        // L, in the pass-1 logits and in the rescored ones.
+        const float E = j <= 0 ? 0.f : __uint_as_float(base + ((uint32_t)j << dec::kBinShift));
+        const float eps = (float)Hq * 0x1p-23f;
+        const float thr = (E - eps) * (8.f / 9.f) * (1.f - 0x1p-10f);
+        const float* srow = lrow + (size_t)b * score_ld;
+        // chunks start on 128-token boundaries; score rows are padded to 4
+        for (int s0 = s_begin + 4 * (int)threadIdx.x; s0 < s_end; s0 += 4 * kGatherThreads) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(srow + s0));
+            const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                if (s0 + i < s_end && e[i] >= thr) {
+                    const unsigned p = atomicAdd(&sh.n_cand, 1u);
+                    if (p < (unsigned)kCandCap) sh.cand[p] = s0 + i;
+                }
+            }
+        }
+        __syncthreads();
+        const int nc = (int)sh.n_cand;
+        if (nc > kCandCap) {
+            if (threadIdx.x == 0) atomicOr(ovf + b, 1u);
+        } else {
+            float l2[16];
+#pragma unroll
+            for (int h = 0; h < 16; h++) l2[h] = h < Hq ? __ldcg(lse2_ws + b * 16 + h) : INFINITY;
+            const uint8_t* kb = kc + (size_t)b * Tmax * 128;
+            const float* ksb = ksc + (size_t)b * Tmax;
+            for (int i0 = warp * 32; i0 < nc; i0 += kGatherThreads) {
+                const int i = i0 + lane;
+                const bool has = i < nc;
+                const int s = has ? sh.cand[i] : 0;
+                uint4 kw[8];
+                const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)s * 128);
+#pragma unroll
+                for (int c = 0; c < 8; c++) kw[c] = has ? __ldg(kr + c) : make_uint4(0u, 0u, 0u, 0u);
+                const float sk = has ? __ldg(ksb + s) : 0.f;
+                float d[16];
+#pragma unroll
+                for (int h = 0; h < 16; h++) d[h] = 0.f;
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    const uint32_t wd[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
+#pragma unroll
+                    for (int m = 0; m < 4; m++) {
+                        const float2 k01 = f16x2_to_float2(e4m3x2_lo_to_f16x2(wd[m]));
+                        const float2 k23 = f16x2_to_float2(e4m3x2_lo_to_f16x2(wd[m] >> 16));
+                        const int dim = 16 * c + 4 * m;
+#pragma unroll
+                        for (int h = 0; h < 16; h++) {
+                            const float4 qv = *reinterpret_cast<const float4*>(&sh.q[h][dim]);
+                            d[h] = fmaf(qv.x, k01.x, d[h]);
+                            d[h] = fmaf(qv.y, k01.y, d[h]);
+                            d[h] = fmaf(qv.z, k23.x, d[h]);
+                            d[h] = fmaf(qv.w, k23.y, d[h]);
+                        }
+                    }
+                }
+                const float ks = sk * qk2;
+                float sc = 0.f;
+#pragma unroll
+                for (int h = 0; h < 16; h++) sc += ex2(fmaf(d[h], ks, -l2[h]));
+                // one boundary-buffer reservation per warp
+                const unsigned m = __ballot_sync(0xffffffffu, has);
+                unsigned basep = 0;
+                if (lane == 0) basep = atomicAdd(bnd_cnt + b, (unsigned)__popc(m));
+                basep = __shfl_sync(0xffffffffu, basep, 0);
+                if (has) {
+                    const unsigned p = basep + (unsigned)__popc(m & ((1u << lane) - 1u));
+                    if (p < (unsigned)dec::BCAP)
+                        bnd[(size_t)b * dec::BCAP + p] = make_key(sc, (uint32_t)s);
+                    else
+                        atomicOr(ovf + b, 1u);
+                }
+            }
+        }
+    } else if (k > 0) {
+        for (int s = s_begin + threadIdx.x; s < s_end; s += blockDim.x) row[wl + s] = s;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) sh.last = (atomicAdd(counter + b, 1u) == (unsigned)(n_chunks - 1));
+    __syncthreads();
+    if (!sh.last) return;
+    __threadfence();
+    const int n_glob = min(k, n_cand);
+    if (ranked) {
+        const unsigned nb_all = __ldcg(bnd_cnt + b);
+        if (__ldcg(ovf + b) != 0u || nb_all < (unsigned)k || nb_all > (unsigned)dec::BCAP) {
+            // the exact pass and its gather write this sequence's row
+            if (threadIdx.x == 0) atomicOr(ovf + b, 1u);
+            return;
+        }
+        const int nb = (int)nb_all;
+        for (int i = threadIdx.x; i < nb; i += blockDim.x)
+            skeys[i] = __ldcg(bnd + (size_t)b * dec::BCAP + i);
+        __syncthreads();
+        const uint64_t thr = block_radix_threshold([&](int i) { return skeys[i]; }, nb, k, sh.hist);
+        __syncthreads();
+        for (int i = threadIdx.x; i < nb; i += blockDim.x)
+            if (skeys[i] >= thr) row[wl + atomicAdd(out_cnt + b, 1u)] = (int32_t)key_pos(skeys[i]);
+    }
+    for (int i = threadIdx.x; i < wl; i += blockDim.x) row[i] = t - wl + 1 + i;
+    for (int i = wl + n_glob + threadIdx.x; i < S; i += blockDim.x) row[i] = -1;
+}
+
+}  // namespace dsk
+}  // namespace hs2

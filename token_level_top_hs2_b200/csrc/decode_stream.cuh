@@ -375,10 +375,12 @@ gather_kernel(const float* __restrict__ scores, int score_ld, const unsigned* __
               const int32_t* __restrict__ lengths, int Tmax, int Hq, int W, int k,
               int chunk_len, int n_chunks, unsigned* __restrict__ out_cnt,
               unsigned* __restrict__ bnd_cnt, uint64_t* __restrict__ bnd,
-              unsigned* __restrict__ counter, int32_t* __restrict__ idx) {
+              unsigned* __restrict__ counter, int32_t* __restrict__ idx,
+              const unsigned* __restrict__ gate) {
     extern __shared__ uint64_t sk[];  // BCAP keys (last CTA)
     __shared__ GatherShared sh;
     const int b = blockIdx.y, chunk = blockIdx.x;
+    if (gate != nullptr && __ldg(gate + b) == 0u) return;
     const int T = __ldg(lengths + b);
     const bool ok = T >= 1 && T <= Tmax;
     const int n_cand = ok ? max(0, T - W) : 0;

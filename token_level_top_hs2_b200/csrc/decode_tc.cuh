@@ -33,6 +33,10 @@ using namespace hs2::tc;
 constexpr int TOK = 128;
 constexpr int kThreads = 320;
 constexpr float kLazy = 8.f;
+// Softmax reference offset: probabilities are formed against R = max - kSk,
+// so 2^(x - R) lies in (0, 2^14] and its f16 value keeps 3 mantissa bits down
+// to 2^-14 before going subnormal (the sketch's 8-bit code range).
+constexpr float kSk = 6.f;
 constexpr int NRMAX = 12;
 // TMEM columns: S^T buffers, O^T, then the two f16 K tiles (A operand of QK:
 // lane = token, 64 columns of packed f16 pairs = the 128 dims)
@@ -190,6 +194,7 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 int n_chunks, float qk_scale, float* __restrict__ part,
                 unsigned* __restrict__ counter, float* __restrict__ lse2_ws,
                 float* __restrict__ lse_out, __nv_bfloat16* __restrict__ out,
+                uint8_t* __restrict__ sketch, float* __restrict__ rsnap, int sk_tiles,
                 unsigned* __restrict__ flags) {
     constexpr int D = 128;
     constexpr int PART = 16 * D + 32;
@@ -362,10 +367,12 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         const int t = wq * 32 + lane;            // token row = TMEM lane
         const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
         uint8_t* pf = smem + LY::OFF_P;
-        float M[16], l[16];
+        // R = running max - kSk: probabilities are formed as 2^(x - R), in
+        // (0, 2^(kLazy + kSk)], which is the range the sketch codes cover
+        float R[16], l[16];
 #pragma unroll
         for (int h = 0; h < 16; h++) {
-            M[h] = -INFINITY;
+            R[h] = -INFINITY;
             l[h] = 0.f;
         }
         bool ok = true;
@@ -380,7 +387,7 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             tmem_ld16(lane_addr + COL_S + buf * 16, r);
             tmem_ld_wait();
             const float ks = skb[buf * TOK + t] * qk_scale;
-            const float sv = svb[buf * TOK + t];
+            const float sv = svb[buf * TOK + t] * (1.f / 64.f);
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.s_empty[buf]);
@@ -390,7 +397,7 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
             for (int h = 0; h < 16; h++) {
                 x[h] = valid ? __uint_as_float(r[h]) * ks : -INFINITY;
-                over |= x[h] > M[h] + kLazy;
+                over |= x[h] > R[h] + (kLazy + kSk);
             }
             if (bar_red_or(over, 1, 128)) {
                 // raise the per-head running max to this tile's max
@@ -415,10 +422,10 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
                 for (int h = 0; h < 16; h++) {
                     const float tm = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
-                    const float nm = fmaxf(M[h], tm);
-                    alpha[h] = (M[h] == -INFINITY || nm == M[h]) ? 1.f : ex2(M[h] - nm);
+                    const float nm = fmaxf(R[h], tm - kSk);
+                    alpha[h] = (R[h] == -INFINITY || nm == R[h]) ? 1.f : ex2(R[h] - nm);
                     any_scale |= alpha[h] != 1.f;
-                    M[h] = nm;
+                    R[h] = nm;
                     l[h] *= alpha[h];
                 }
                 bar_named(2, 128);  // red[] is read by everyone before it is reused
@@ -440,11 +447,33 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 }
             }
             uint32_t pw[16];
+            float pr[16];
 #pragma unroll
             for (int h = 0; h < 16; h++) {
-                const float p = (valid && M[h] != -INFINITY) ? ex2(x[h] - M[h]) : 0.f;
-                l[h] += p;
-                pw[h] = __half_as_ushort(__float2half_rn(p * sv));
+                pr[h] = (valid && R[h] != -INFINITY) ? ex2(x[h] - R[h]) : 0.f;
+                l[h] += pr[h];
+                pw[h] = __half_as_ushort(__float2half_rn(pr[h] * sv));
+            }
+            if (sketch != nullptr) {
+                const int tok = s_begin + j * TOK + t;
+                if (valid) {
+                    uint32_t hw[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i++) hw[i] = f16x2_rz(pr[2 * i], pr[2 * i + 1]);
+                    uint4 cw;
+                    cw.x = prmt(hw[0] >> 7, hw[1] >> 7, 0x6420u);
+                    cw.y = prmt(hw[2] >> 7, hw[3] >> 7, 0x6420u);
+                    cw.z = prmt(hw[4] >> 7, hw[5] >> 7, 0x6420u);
+                    cw.w = prmt(hw[6] >> 7, hw[7] >> 7, 0x6420u);
+                    *reinterpret_cast<uint4*>(sketch + ((size_t)b * Tmax + tok) * 16) = cw;
+                }
+                if (wq == 0 && lane < 16) {
+                    float rv = R[0];
+#pragma unroll
+                    for (int h = 1; h < 16; h++)
+                        if (lane == h) rv = R[h];
+                    rsnap[((size_t)b * sk_tiles + (s_begin / TOK + j)) * 16 + lane] = rv;
+                }
             }
             if (u > 0 && !mbar_wait(&bars.p_empty[buf], (u - 1) & 1, abort_, flags)) {
                 ok = false;
@@ -476,12 +505,14 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         bar_named(2, 128);
         float* dst = part + ((size_t)b * n_chunks + chunk) * PART;
         if (t < 16) {
-            float mt = M[0];
+            float mt = R[0];
 #pragma unroll
             for (int h = 1; h < 16; h++)
-                if (t == h) mt = M[h];
-            dst[16 * D + t] = mt;
-            dst[16 * D + 16 + t] = red[t] + red[16 + t] + red[32 + t] + red[48 + t];
+                if (t == h) mt = R[h];
+            // O is relative to R + kSk (the P tiles carry sv / 64), so is the sum
+            dst[16 * D + t] = mt + kSk;
+            dst[16 * D + 16 + t] =
+                (red[t] + red[16 + t] + red[32 + t] + red[48 + t]) * (1.f / 64.f);
         }
         if (ok && n > 0 && mbar_wait(&bars.o_done, (n - 1) & 1, abort_, flags)) {
             fence_after_sync();
@@ -532,13 +563,14 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 }
 
 // ----------------------------------------------------------------------------
-// Pass 2: the candidates' scores and the per-sequence histogram.
+// Pass 2: the candidates' exact scores and the per-sequence histogram (the
+// fallback of the sketch selection, for sequences flagged in `gate`).
 __global__ void __launch_bounds__(kThreads, 1)
 pass2_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_ks,
                 const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ lengths, int Tmax,
                 int Hq, int W, int chunk_len, float qk_scale, const float* __restrict__ lse2_ws,
                 float* __restrict__ scores, int score_ld, unsigned* __restrict__ hist_g,
-                unsigned* __restrict__ flags) {
+                const unsigned* __restrict__ gate, unsigned* __restrict__ flags) {
     constexpr int D = 128;
     using LY = Layout<false>;
     constexpr int NR = LY::NR;
@@ -548,6 +580,8 @@ pass2_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     __shared__ Bars bars;
     __shared__ unsigned hist[256];
     const int b = blockIdx.y, chunk = blockIdx.x;
+    // run only for the sequences the sketch selection handed over, if gated
+    if (gate != nullptr && __ldg(gate + b) == 0u) return;
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int T = __ldg(lengths + b);
     const int n_cand = (T >= 1 && T <= Tmax) ? max(0, T - W) : 0;

@@ -12,6 +12,7 @@
 #include "../../include/hs2.h"
 #include "decode_kernels.cuh"
 #include "decode_stream.cuh"
+#include "decode_sketch.cuh"
 #include "decode_tc.cuh"
 #include "prefill_kernels.cuh"
 #include "prefill_tc.cuh"
@@ -80,7 +81,9 @@ std::mutex g_smem_mutex;
 
 template <class K>
 bool set_smem(K kernel, size_t bytes) {
-    if (bytes <= 48 * 1024) return true;
+    // (static + dynamic shared memory above 48 KiB needs the opt-in, so any
+    // nonzero request is registered; the table makes it once per kernel/device)
+    if (bytes == 0) return true;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     const void* fn = reinterpret_cast<const void*>(kernel);
@@ -288,9 +291,15 @@ bool decode_streamable(const hs2_decode_shape* s) {
 }
 
 struct DecodeWs2 {
-    int n_chunks, chunk_len, score_ld;
-    size_t zero_off, zero_bytes, lse2_off, part_off, score_off, bnd_off, total;
+    int n_chunks, chunk_len, score_ld, sk_tiles;
+    size_t zero_off, zero_bytes, lse2_off, part_off, score_off, bnd_off, sketch_off, rsnap_off,
+        total;
 };
+
+// The sketch selection (FP8 cache, d = 128, k > 0) replaces the exact pass 2.
+bool decode_uses_sketch(const hs2_decode_shape* s) {
+    return s->kv == HS2_KV_E4M3 && s->d == 128 && s->k > 0;
+}
 DecodeWs2 decode_ws2(const hs2_decode_shape* s) {
     DecodeWs2 w;
     const size_t B = s->B;
@@ -303,15 +312,25 @@ DecodeWs2 decode_ws2(const hs2_decode_shape* s) {
     w.n_chunks = (s->Tmax + w.chunk_len - 1) / w.chunk_len;
     const size_t part_floats = (size_t)16 * s->d + 32;
     size_t off = 0;
-    // zeroed per call: pass-1 counter, gather counter, out count, boundary count, histogram
+    // zeroed per call: pass-1 counter, gather counter, out count, boundary count,
+    // histogram; then the sketch selection's counter, out count, boundary
+    // count, overflow flag and histogram
     w.zero_off = off;
-    w.zero_bytes = B * (4 + 256) * sizeof(unsigned);
+    w.zero_bytes = B * (8 + 512) * sizeof(unsigned);
     off = round_up(off + w.zero_bytes, 256);
     w.lse2_off = off;  off = round_up(off + B * 16 * sizeof(float), 256);
     w.part_off = off;  off = round_up(off + B * w.n_chunks * part_floats * sizeof(float), 256);
     w.score_ld = (s->Tmax + 3) / 4 * 4;  // 16-byte rows
     w.score_off = off; off = round_up(off + B * (size_t)w.score_ld * sizeof(float), 256);
     w.bnd_off = off;   off = round_up(off + B * dec::BCAP * sizeof(uint64_t), 256);
+    w.sk_tiles = (s->Tmax + dec::TOK - 1) / dec::TOK;
+    w.sketch_off = off;
+    w.rsnap_off = off;
+    if (decode_uses_sketch(s)) {
+        off = round_up(off + B * (size_t)s->Tmax * 16, 256);
+        w.rsnap_off = off;
+        off = round_up(off + B * (size_t)w.sk_tiles * 16 * sizeof(float), 256);
+    }
     w.total = off;
     return w;
 }
@@ -332,11 +351,17 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     unsigned* out_cnt = zero + 2 * B;
     unsigned* bnd_cnt = zero + 3 * B;
     unsigned* hist = zero + 4 * B;
+    unsigned* sk_cnt = zero + 260 * B;
+    unsigned* sk_out = zero + 261 * B;
+    unsigned* sk_bnd = zero + 262 * B;
+    unsigned* sk_ovf = zero + 263 * B;
+    unsigned* sk_hist = zero + 264 * B;
     float* lse2 = reinterpret_cast<float*>(ws + w.lse2_off);
     float* part = reinterpret_cast<float*>(ws + w.part_off);
     float* scores = reinterpret_cast<float*>(ws + w.score_off);
     uint64_t* bnd = reinterpret_cast<uint64_t*>(ws + w.bnd_off);
     const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
+    const unsigned* gate = nullptr;
     CUtensorMap mk, mv, mks, mvs;
     if (!map_cache(&mk, kc, s->B, s->Tmax, D, FP8) || !map_cache(&mv, vc, s->B, s->Tmax, D, FP8))
         return HS2_ERR_CUDA;
@@ -354,18 +379,36 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
         const float qk2 = s->scale * kLog2e;
         using LY = dtc::Layout<true>;
         using LY2 = dtc::Layout<false>;
+        const bool sketch = decode_uses_sketch(s);
+        uint8_t* skt = sketch ? ws + w.sketch_off : nullptr;
+        float* rsnap = reinterpret_cast<float*>(ws + w.rsnap_off);
         if (!set_smem(dtc::pass1_tc_kernel, LY::SMEM)) return HS2_ERR_CUDA;
         dtc::pass1_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kThreads, LY::SMEM, st>>>(
             mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len, w.n_chunks, qk2, part,
-            cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), flags);
+            cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), skt, rsnap, w.sk_tiles, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-        if (s->k > 0) {
+        if (sketch) {
+            // three resident CTAs per SM over the whole batch, one wave
+            const int g_sc = 3 * 148 / s->B > 0 ? 3 * 148 / s->B : 1;
+            dsk::sketch_score_kernel<<<dim3(g_sc, s->B), dsk::kScoreThreads, 0, st>>>(
+                skt, rsnap, w.sk_tiles, lengths, s->Tmax, s->Hq, s->W, s->k, lse2, scores,
+                w.score_ld, sk_hist);
+            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+            const size_t smem = (size_t)dec::BCAP * sizeof(uint64_t);
+            if (!set_smem(dsk::sketch_gather_kernel, smem)) return HS2_ERR_CUDA;
+            dsk::sketch_gather_kernel<<<dim3(w.n_chunks, s->B), dsk::kGatherThreads, smem, st>>>(
+                scores, w.score_ld, sk_hist, static_cast<const uint8_t*>(kc), ks, qp, lse2, qk2,
+                lengths, s->Tmax, s->Hq, s->W, s->k, w.chunk_len, w.n_chunks, sk_bnd, bnd, sk_ovf,
+                sk_cnt, sk_out, idx);
+            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+            // sequences whose candidates overflowed: exact scores, then the exact gather
             if (!set_smem(dtc::pass2_tc_kernel, LY2::SMEM)) return HS2_ERR_CUDA;
             dtc::pass2_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kThreads, LY2::SMEM, st>>>(
                 mk, mks, qp, lengths, s->Tmax, s->Hq, s->W, w.chunk_len, qk2, lse2, scores,
-                w.score_ld, hist, flags);
+                w.score_ld, hist, sk_ovf, flags);
             if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
         }
+        gate = sketch ? sk_ovf : nullptr;
     } else {
         auto kern = dec::pass1_kernel<D, FP8>;
         if (!set_smem(kern, SG::SMEM1)) return HS2_ERR_CUDA;
@@ -387,8 +430,7 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
         if (!set_smem(dec::gather_kernel, smem)) return HS2_ERR_CUDA;
         dec::gather_kernel<<<dim3(w.n_chunks, s->B), 256, smem, st>>>(
             scores, w.score_ld, hist, lengths, s->Tmax, s->Hq, s->W, s->k, w.chunk_len, w.n_chunks,
-            out_cnt,
-            bnd_cnt, bnd, cnt3, idx);
+            out_cnt, bnd_cnt, bnd, cnt3, idx, gate);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     return HS2_OK;
