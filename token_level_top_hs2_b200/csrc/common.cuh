@@ -230,6 +230,16 @@ HS2_DEV int warp_find_bin(const int* hist, int need, int* above_out, int* in_bin
 // of keys[0..n) are >= T (requires 0 < kk <= n).  Most-significant 8-bit digit
 // first; stops as soon as the keys sharing the selected prefix are all taken.
 //
+// One histogram update per distinct digit of the warp (candidate keys share
+// their leading digits, so per-key atomics would serialise on one bin).  All
+// 32 lanes call it.
+HS2_DEV void count_digit(int* hist, uint64_t key, bool in, uint64_t mask, uint64_t prefix,
+                         int shift) {
+    const int d = (in && (key & mask) == prefix) ? (int)((key >> shift) & 255) : -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, d);
+    if (d >= 0 && lane_id() == __ffs(grp) - 1) atomicAdd(&hist[d], __popc(grp));
+}
+
 // Warp version: one warp, hist = 256 ints of shared memory owned by the warp.
 template <class Get>
 HS2_DEV uint64_t warp_radix_threshold(Get get, int n, int kk, int* hist) {
@@ -240,9 +250,9 @@ HS2_DEV uint64_t warp_radix_threshold(Get get, int n, int kk, int* hist) {
 #pragma unroll
         for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
         __syncwarp();
-        for (int i = lane; i < n; i += 32) {
-            uint64_t key = get(i);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        for (int i0 = 0; i0 < n; i0 += 32) {
+            count_digit(hist, i0 + lane < n ? get(i0 + lane) : 0, i0 + lane < n, mask, prefix,
+                        shift);
         }
         __syncwarp();
         // lane owns digits 8*lane .. 8*lane+7; suffix sums from the top digit down
@@ -296,9 +306,9 @@ HS2_DEV uint64_t block_radix_threshold(Get get, int n, int kk, int* hist) {
     for (int shift = 56; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < n; i += blockDim.x) {
-            uint64_t key = get(i);
-            if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255], 1);
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+            const int i = i0 + tid;
+            count_digit(hist, i < n ? get(i) : 0, i < n, mask, prefix, shift);
         }
         __syncthreads();
         if (tid < 32) {

@@ -1,0 +1,491 @@
+// Decode pass 1 on the tensor cores (FP8 e4m3 cache, d = 128): exact lse and
+// O of one query per sequence over a chunk of its cache, plus the per-token
+// selection sketch (decode_sketch.cuh).
+//
+// HySparse2 summary (onedev.kr/papers/146), 'How it works': the full layer is
+// exact attention; each cached row is dequantised as s_x * e4m3(x) with its
+// per-token scale.  The e4m3 -> f16 conversion is exact, and the scales are
+// folded in afterwards (logit * sK, p * sV), so the MMAs see exact operands.
+//
+// Per 128-token tile, with the tokens as the MMA M dimension:
+//   S^T[token][head] = K_tile (128 x 128, f16, TMEM) * Q^T (128 x 16, f16)
+//   O^T[dim][head]  += V_tile^T (128 x 128, f16, smem) * P (128 x 16, f16)
+// Roles (12 warps):
+//   warp 0       TMA producer: raw e4m3 K, V tiles and both scale rows into a
+//                ring of kNR stages;
+//   warp 1       MMA issuer: a non-blocking scheduler that issues whichever of
+//                QK(next) / PV(next) has its operands ready, so a tile's QK
+//                never waits behind an older tile's PV;
+//   warps 2-5    K converters: thread = token row = TMEM lane; e4m3 -> f16
+//                straight into one of kDK TMEM K buffers; copy both scales;
+//   warps 6-9    softmax: thread = token = TMEM lane of S^T; lazily raised
+//                CTA-wide running max; P (f16, K-major) into one of kDV shared
+//                buffers; the per-token sketch bytes;
+//   warps 10-11  V converters: two token rows per thread, e4m3 -> f16 into one
+//                of kDV shared V tiles (canonical 128-byte-swizzled layout).
+// K and V conversion run in separate warps so that the QK/softmax chain of
+// later tiles proceeds while an older tile's PV is still pending.
+#pragma once
+
+#include "decode_tc.cuh"
+
+namespace hs2 {
+namespace dtc {
+
+constexpr int kP1Threads = 384;
+constexpr int kNR = 4;  // raw stages
+constexpr int kDK = 4;  // K tiles in TMEM = S^T buffers = scale slots
+constexpr int kDV = 2;  // f16 V tiles and P tiles in shared memory
+// TMEM columns (512 allocated, one CTA per SM): S^T buffers, O^T, K tiles
+constexpr uint32_t P1_COL_S = 0, P1_COL_O = 16 * kDK, P1_COL_K = 128;
+static_assert(P1_COL_O + 16 <= P1_COL_K && P1_COL_K + 64 * kDK <= 512, "TMEM plan");
+
+struct P1Layout {
+    static constexpr int RAW_K = 0, RAW_V = TOK * 128;
+    static constexpr int RAW_SK = 2 * TOK * 128, RAW_SV = RAW_SK + TOK * 4;
+    static constexpr int RAW = 34816;                      // stage stride, 1024-aligned
+    static constexpr int F16T = 2 * TOK * 128;             // f16 V tile
+    static constexpr int PT = 2 * 16 * 128;                // P tile: 2 blocks of 16 x 128 B
+    static constexpr int OFF_RAW = 0;
+    static constexpr int OFF_VF = OFF_RAW + kNR * RAW;
+    static constexpr int OFF_QF = OFF_VF + kDV * F16T;
+    static constexpr int OFF_P = OFF_QF + PT;
+    static constexpr int OFF_SC = OFF_P + kDV * PT;        // sk[kDK][128], sv[kDK][128]
+    static constexpr int OFF_RED = OFF_SC + 2 * kDK * TOK * 4;  // [4][16] floats
+    static constexpr int SMEM = OFF_RED + 4 * 16 * 4 + 1024;
+    static_assert(RAW >= RAW_SV + TOK * 4 && RAW % 1024 == 0, "raw stage");
+    static_assert(OFF_VF % 1024 == 0 && OFF_QF % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+struct P1Bars {
+    uint64_t raw_full[kNR], raw_empty[kNR];
+    uint64_t q_ready, kf_full[kDK], kf_empty[kDK], s_full[kDK], s_empty[kDK];
+    uint64_t vf_full[kDV], vf_empty[kDV], p_full[kDV], p_empty[kDV], drain;
+    uint32_t tmem_base;
+    int abort_;
+    unsigned last;
+};
+
+// Spin guard of the MMA scheduler: after kWaitNs without progress it raises
+// the abort flag (everybody's bounded waits then give up) and FLAG_TIMEOUT.
+struct SpinGuard {
+    uint64_t t0 = 0;
+    uint32_t i = 0;
+    HS2_DEV void progress() { i = 0; t0 = 0; }
+    HS2_DEV bool idle(volatile int* abort_, unsigned* flags) {
+        if ((++i & 255u) != 0) return true;
+        if (*abort_) return false;
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        if (now - t0 > kWaitNs) {
+            *abort_ = 1;
+            atomicOr(flags, FLAG_TIMEOUT);
+            return false;
+        }
+        return true;
+    }
+};
+
+HS2_DEV void p1_issue_raw(uint8_t* st, const CUtensorMap* mk, const CUtensorMap* mv,
+                          const CUtensorMap* mks, const CUtensorMap* mvs, int tok, int b,
+                          uint64_t* bar) {
+    mbar_arrive_expect_tx(bar, 2 * (TOK * 128 + TOK * 4));
+    tma_load_3d(st + P1Layout::RAW_K, mk, 0, tok, b, bar);
+    tma_load_3d(st + P1Layout::RAW_V, mv, 0, tok, b, bar);
+    tma_load_2d(st + P1Layout::RAW_SK, mks, tok, b, bar);
+    tma_load_2d(st + P1Layout::RAW_SV, mvs, tok, b, bar);
+}
+
+// grid (n_chunks, B), 384 threads; the last chunk of a sequence to finish
+// merges every chunk's partial into O and lse.
+__global__ void __launch_bounds__(kP1Threads, 1)
+pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                const __grid_constant__ CUtensorMap map_ks,
+                const __grid_constant__ CUtensorMap map_vs, const __nv_bfloat16* __restrict__ q,
+                const int32_t* __restrict__ lengths, int Tmax, int Hq, int chunk_len,
+                int n_chunks, float qk_scale, float* __restrict__ part,
+                unsigned* __restrict__ counter, float* __restrict__ lse2_ws,
+                float* __restrict__ lse_out, __nv_bfloat16* __restrict__ out,
+                uint8_t* __restrict__ sketch, float* __restrict__ rsnap, int sk_tiles,
+                unsigned* __restrict__ flags) {
+    constexpr int D = 128;
+    constexpr int PART = 16 * D + 32;
+    using LY = P1Layout;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    __shared__ P1Bars bars;
+    const int b = blockIdx.y, chunk = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    const int T = __ldg(lengths + b);
+    const bool len_ok = T >= 1 && T <= Tmax;
+    if (!len_ok && threadIdx.x == 0 && chunk == 0) atomicOr(flags, FLAG_BAD_LENGTH);
+    const int s_begin = chunk * chunk_len;
+    const int s_end = len_ok ? min(s_begin + chunk_len, T) : s_begin;
+    const int n = s_end > s_begin ? (s_end - s_begin + TOK - 1) / TOK : 0;
+    volatile int* abort_ = &bars.abort_;
+    float* skb = reinterpret_cast<float*>(smem + LY::OFF_SC);  // [kDK][128]
+    float* svb = skb + kDK * TOK;                              // [kDK][128]
+    float* red = reinterpret_cast<float*>(smem + LY::OFF_RED); // [4][16]
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNR; i++) {
+            mbar_init(&bars.raw_full[i], 1);
+            mbar_init(&bars.raw_empty[i], 6);  // 4 K-converter + 2 V-converter warps
+        }
+        mbar_init(&bars.q_ready, 4);
+        for (int i = 0; i < kDK; i++) {
+            mbar_init(&bars.kf_full[i], 4);
+            mbar_init(&bars.kf_empty[i], 1);
+            mbar_init(&bars.s_full[i], 1);
+            mbar_init(&bars.s_empty[i], 4);
+        }
+        for (int i = 0; i < kDV; i++) {
+            mbar_init(&bars.vf_full[i], 2);
+            mbar_init(&bars.vf_empty[i], 1);
+            mbar_init(&bars.p_full[i], 4);
+            mbar_init(&bars.p_empty[i], 1);
+        }
+        mbar_init(&bars.drain, 1);
+        bars.abort_ = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bars.tmem_base, 512);
+        tmem_relinquish();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = bars.tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0 && n > 0) {
+            // ------------------------------------------------------ producer
+            int armed = 0;
+            for (int j = 0; j < n && !*abort_; j++) {
+                const int st = j % kNR, u = j / kNR;
+                if (u > 0 && !mbar_wait(&bars.raw_empty[st], (u - 1) & 1, abort_, flags)) break;
+                p1_issue_raw(smem + LY::OFF_RAW + st * LY::RAW, &map_k, &map_v, &map_ks, &map_vs,
+                             s_begin + j * TOK, b, &bars.raw_full[st]);
+                armed++;
+            }
+            if (*abort_) {
+                volatile int no_abort = 0;
+                for (int j = max(0, armed - kNR); j < armed; j++)
+                    mbar_wait(&bars.raw_full[j % kNR], (j / kNR) & 1, &no_abort, flags);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && n > 0) {
+            // --------------------------------------------- MMA scheduler
+            constexpr uint32_t id_qk = idesc_f16(128, 16, false, false);
+            constexpr uint32_t id_pv = idesc_f16(128, 16, true, false);
+            const uint32_t vf = smem_u32(smem + LY::OFF_VF);
+            const uint32_t qf = smem_u32(smem + LY::OFF_QF), pf = smem_u32(smem + LY::OFF_P);
+            bool ok = mbar_wait(&bars.q_ready, 0, abort_, flags);
+            int nq = 0, np = 0;  // next QK / PV tile
+            SpinGuard guard;
+            while (ok && np < n) {
+                const int vb = np % kDV, vu = np / kDV;
+                if (np < nq && mbar_try_wait(&bars.p_full[vb], vu & 1) &&
+                    mbar_try_wait(&bars.vf_full[vb], vu & 1)) {
+                    fence_after_sync();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ks++) {
+                        const uint32_t va = vf + vb * LY::F16T + ks * (16 * 128);
+                        const uint32_t pb = pf + vb * LY::PT + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
+                        mma_ss(tmem + P1_COL_O, sdesc_sw128(va, TOK * 128, 1024),
+                               sdesc_sw128(pb, 16, 1024), id_pv, (np > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&bars.vf_empty[vb]);
+                    mma_commit(&bars.p_empty[vb]);
+                    np++;
+                    guard.progress();
+                    continue;
+                }
+                const int kb = nq % kDK, ku = nq / kDK;
+                if (nq < n && mbar_try_wait(&bars.kf_full[kb], ku & 1) &&
+                    (ku == 0 || mbar_try_wait(&bars.s_empty[kb], (ku - 1) & 1))) {
+                    fence_after_sync();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ks++) {
+                        const uint32_t kbq = qf + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
+                        mma_ts(tmem + P1_COL_S + kb * 16, tmem + P1_COL_K + kb * 64 + ks * 8,
+                               sdesc_sw128(kbq, 16, 1024), id_qk, ks > 0);
+                    }
+                    mma_commit(&bars.s_full[kb]);
+                    mma_commit(&bars.kf_empty[kb]);
+                    nq++;
+                    guard.progress();
+                    continue;
+                }
+                ok = guard.idle(abort_, flags);
+            }
+            mma_commit(&bars.drain);
+            volatile int no_abort = 0;
+            mbar_wait(&bars.drain, 0, &no_abort, flags);
+        }
+    } else if (warp < 6) {
+        // ---------------------------------------------------- K converters
+        const int t = (warp & 3) * 32 + lane;  // token row = TMEM lane of this warp
+        const uint32_t k_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16) + P1_COL_K;
+        const bool qok = convert_q(q + (size_t)b * Hq * D, Hq, smem + LY::OFF_QF, t);
+        if (!__all_sync(0xffffffffu, qok) && lane == 0 && chunk == 0) atomicOr(flags, FLAG_Q_RANGE);
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.q_ready);
+        bool bad_scale = false;
+        for (int j = 0; j < n; j++) {
+            const int st = j % kNR, kb = j % kDK, ku = j / kDK;
+            if (!mbar_wait(&bars.raw_full[st], (j / kNR) & 1, abort_, flags)) break;
+            // slot kb last held tile j - kDK: its QK must be done and the
+            // softmax must have read its scores and scales
+            if (ku > 0 && (!mbar_wait(&bars.kf_empty[kb], (ku - 1) & 1, abort_, flags) ||
+                           !mbar_wait(&bars.s_empty[kb], (ku - 1) & 1, abort_, flags)))
+                break;
+            const uint8_t* raw = smem + LY::OFF_RAW + st * LY::RAW;
+            const bool valid = s_begin + j * TOK + t < s_end;
+            fence_after_sync();
+            convert_row_tmem(raw + LY::RAW_K, t, valid, k_lane + kb * 64);
+            const float sk = reinterpret_cast<const float*>(raw + LY::RAW_SK)[t];
+            const float sv = reinterpret_cast<const float*>(raw + LY::RAW_SV)[t];
+            skb[kb * TOK + t] = valid ? sk : 0.f;
+            svb[kb * TOK + t] = valid ? sv : 0.f;
+            bad_scale |= valid && !(sv <= 255.f);
+            tmem_st_wait();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars.kf_full[kb]);
+                mbar_arrive(&bars.raw_empty[st]);
+            }
+        }
+        if (__any_sync(0xffffffffu, bad_scale) && lane == 0) atomicOr(flags, FLAG_SCALE_RANGE);
+    } else if (warp >= 10) {
+        // ---------------------------------------------------- V converters
+        const int v = (warp - 10) * 32 + lane;  // rows v and v + 64
+        for (int j = 0; j < n; j++) {
+            const int st = j % kNR, vb = j % kDV, vu = j / kDV;
+            if (!mbar_wait(&bars.raw_full[st], (j / kNR) & 1, abort_, flags)) break;
+            if (vu > 0 && !mbar_wait(&bars.vf_empty[vb], (vu - 1) & 1, abort_, flags)) break;
+            const uint8_t* raw = smem + LY::OFF_RAW + st * LY::RAW + LY::RAW_V;
+            uint8_t* dst = smem + LY::OFF_VF + vb * LY::F16T;
+            const int row0 = s_begin + j * TOK;
+            convert_row(raw, dst, v, row0 + v < s_end);
+            convert_row(raw, dst, v + 64, row0 + v + 64 < s_end);
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bars.vf_full[vb]);
+                mbar_arrive(&bars.raw_empty[st]);
+            }
+        }
+    } else {
+        // ----------------------------------------------------------- softmax
+        const int wq = warp & 3;                 // TMEM lane quarter of this warp
+        const int t = wq * 32 + lane;            // token row = TMEM lane
+        const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
+        uint8_t* pf = smem + LY::OFF_P;
+        // R = running max - kSk: probabilities are formed as 2^(x - R), in
+        // (0, 2^(kLazy + kSk)], which is the range the sketch codes cover
+        float R[16], l[16];
+#pragma unroll
+        for (int h = 0; h < 16; h++) {
+            R[h] = -INFINITY;
+            l[h] = 0.f;
+        }
+        bool ok = true;
+        for (int j = 0; j < n; j++) {
+            const int kb = j % kDK, vb = j % kDV, vu = j / kDV;
+            if (!mbar_wait(&bars.s_full[kb], (j / kDK) & 1, abort_, flags)) {
+                ok = false;
+                break;
+            }
+            fence_after_sync();
+            uint32_t r[16];
+            tmem_ld16(lane_addr + P1_COL_S + kb * 16, r);
+            tmem_ld_wait();
+            const float ks = skb[kb * TOK + t] * qk_scale;
+            const float sv = svb[kb * TOK + t] * (1.f / 64.f);
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.s_empty[kb]);
+            const bool valid = s_begin + j * TOK + t < s_end;
+            float x[16];
+            bool over = false;
+#pragma unroll
+            for (int h = 0; h < 16; h++) {
+                x[h] = valid ? __uint_as_float(r[h]) * ks : -INFINITY;
+                over |= x[h] > R[h] + (kLazy + kSk);
+            }
+            if (bar_red_or(over, 1, 128)) {
+                // raise the per-head running max to this tile's max
+                float mx[16];
+#pragma unroll
+                for (int h = 0; h < 16; h++) {
+                    float v = x[h];
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    mx[h] = v;
+                }
+                if (lane < 16) {
+                    float v = mx[0];
+#pragma unroll
+                    for (int h = 1; h < 16; h++)
+                        if (lane == h) v = mx[h];
+                    red[wq * 16 + lane] = v;
+                }
+                bar_named(2, 128);
+                float alpha[16];
+                bool any_scale = false;
+#pragma unroll
+                for (int h = 0; h < 16; h++) {
+                    const float tm = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
+                    const float nm = fmaxf(R[h], tm - kSk);
+                    alpha[h] = (R[h] == -INFINITY || nm == R[h]) ? 1.f : ex2(R[h] - nm);
+                    any_scale |= alpha[h] != 1.f;
+                    R[h] = nm;
+                    l[h] *= alpha[h];
+                }
+                bar_named(2, 128);  // red[] is read by everyone before it is reused
+                if (j > 0 && any_scale) {
+                    // O^T holds tiles 0..j-1: wait for PV(j-1), scale its columns
+                    const int pb = (j - 1) % kDV, pu = (j - 1) / kDV;
+                    if (!mbar_wait(&bars.p_empty[pb], pu & 1, abort_, flags)) {
+                        ok = false;
+                        break;
+                    }
+                    fence_after_sync();
+                    uint32_t o[16];
+                    tmem_ld16(lane_addr + P1_COL_O, o);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int h = 0; h < 16; h++) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                    tmem_st16(lane_addr + P1_COL_O, o);
+                    tmem_st_wait();
+                    fence_before_sync();
+                }
+            }
+            uint32_t pw[16];
+            float pr[16];
+#pragma unroll
+            for (int h = 0; h < 16; h++) {
+                pr[h] = (valid && R[h] != -INFINITY) ? ex2(x[h] - R[h]) : 0.f;
+                l[h] += pr[h];
+                pw[h] = __half_as_ushort(__float2half_rn(pr[h] * sv));
+            }
+            if (sketch != nullptr) {
+                const int tok = s_begin + j * TOK + t;
+                if (valid) {
+                    uint32_t hw[8];
+#pragma unroll
+                    for (int i = 0; i < 8; i++) hw[i] = f16x2_rz(pr[2 * i], pr[2 * i + 1]);
+                    uint4 cw;
+                    cw.x = prmt(hw[0] >> 7, hw[1] >> 7, 0x6420u);
+                    cw.y = prmt(hw[2] >> 7, hw[3] >> 7, 0x6420u);
+                    cw.z = prmt(hw[4] >> 7, hw[5] >> 7, 0x6420u);
+                    cw.w = prmt(hw[6] >> 7, hw[7] >> 7, 0x6420u);
+                    *reinterpret_cast<uint4*>(sketch + ((size_t)b * Tmax + tok) * 16) = cw;
+                }
+                if (wq == 0 && lane < 16) {
+                    float rv = R[0];
+#pragma unroll
+                    for (int h = 1; h < 16; h++)
+                        if (lane == h) rv = R[h];
+                    rsnap[((size_t)b * sk_tiles + (s_begin / TOK + j)) * 16 + lane] = rv;
+                }
+            }
+            if (vu > 0 && !mbar_wait(&bars.p_empty[vb], (vu - 1) & 1, abort_, flags)) {
+                ok = false;
+                break;
+            }
+            uint8_t* pt = pf + vb * LY::PT;
+#pragma unroll
+            for (int h = 0; h < 16; h++)
+                *reinterpret_cast<uint16_t*>(pt + f16_off(16, h, t)) = (uint16_t)pw[h];
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars.p_full[vb]);
+        }
+        // chunk partial: l summed over the tile rows, O^T from TMEM (lane = dim)
+#pragma unroll
+        for (int h = 0; h < 16; h++) {
+            float v = l[h];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            l[h] = v;
+        }
+        if (lane < 16) {
+            float v = l[0];
+#pragma unroll
+            for (int h = 1; h < 16; h++)
+                if (lane == h) v = l[h];
+            red[wq * 16 + lane] = v;
+        }
+        bar_named(2, 128);
+        float* dst = part + ((size_t)b * n_chunks + chunk) * PART;
+        if (t < 16) {
+            float mt = R[0];
+#pragma unroll
+            for (int h = 1; h < 16; h++)
+                if (t == h) mt = R[h];
+            // O is relative to R + kSk (the P tiles carry sv / 64), so is the sum
+            dst[16 * D + t] = mt + kSk;
+            dst[16 * D + 16 + t] =
+                (red[t] + red[16 + t] + red[32 + t] + red[48 + t]) * (1.f / 64.f);
+        }
+        // the last PV (and with it every earlier one) has completed once its
+        // P buffer is released
+        if (ok && n > 0 &&
+            mbar_wait(&bars.p_empty[(n - 1) % kDV], ((n - 1) / kDV) & 1, abort_, flags)) {
+            fence_after_sync();
+            uint32_t o[16];
+            tmem_ld16(lane_addr + P1_COL_O, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int h = 0; h < 16; h++) dst[h * D + t] = __uint_as_float(o[h]);
+        } else {
+#pragma unroll
+            for (int h = 0; h < 16; h++) dst[h * D + t] = 0.f;
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+    // ---- the last chunk of the sequence merges every chunk's partial
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) bars.last = (atomicAdd(counter + b, 1u) == (unsigned)(n_chunks - 1));
+    __syncthreads();
+    if (!bars.last) return;
+    __threadfence();
+    const float* pb = part + (size_t)b * n_chunks * PART;
+    for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
+        const int row = e / D;
+        float mx = -INFINITY;
+        for (int i = 0; i < n_chunks; i++)
+            mx = fmaxf(mx, __ldcg(pb + (size_t)i * PART + 16 * D + row));
+        const float mu = mx == -INFINITY ? 0.f : mx;
+        float acc = 0.f, ls = 0.f;
+        for (int i = 0; i < n_chunks; i++) {
+            const float* p = pb + (size_t)i * PART;
+            const float f = ex2(__ldcg(p + 16 * D + row) - mu);
+            acc += f * __ldcg(p + e);
+            ls += f * __ldcg(p + 16 * D + 16 + row);
+        }
+        out[(size_t)b * Hq * D + e] = __float2bfloat16_rn(ls > 0.f ? acc / ls : 0.f);
+        if (e % D == 0) {
+            const float l2 = ls > 0.f ? mu + __log2f(ls) : -INFINITY;
+            lse2_ws[b * 16 + row] = l2;
+            if (lse_out) lse_out[b * Hq + row] = l2 * kLn2;
+        }
+    }
+}
+
+}  // namespace dtc
+}  // namespace hs2

@@ -48,12 +48,13 @@ sketch_score_kernel(const uint8_t* __restrict__ sketch, const float* __restrict_
                     int sk_tiles, const int32_t* __restrict__ lengths, int Tmax, int Hq, int W,
                     int k, const float* __restrict__ lse2_ws, float* __restrict__ lrow,
                     int score_ld, unsigned* __restrict__ hist_g) {
-    __shared__ unsigned hist[256];
+    // one counter column per lane: the lanes of a warp never collide
+    __shared__ unsigned hist[256 * 32];
     const int b = blockIdx.y;
     const int T = __ldg(lengths + b);
     const int n_cand = (T >= 1 && T <= Tmax) ? max(0, T - W) : 0;
     if (k <= 0 || n_cand <= k) return;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = lane_id();
     constexpr int NW = kScoreThreads / 32;
@@ -103,17 +104,19 @@ sketch_score_kernel(const uint8_t* __restrict__ sketch, const float* __restrict_
                     L = fmaf(w[4 * i + 2], c.x, L);
                     L = fmaf(w[4 * i + 3], c.y, L);
                 }
-                const bool valid = tok < n_cand;
-                if (valid) srow[tok] = L;
-                const int bn = valid ? dec::score_bin(__float_as_uint(L), base) : -1;
-                const unsigned grp = __match_any_sync(0xffffffffu, bn);
-                if (valid && lane == __ffs(grp) - 1) atomicAdd(&hist[bn], (unsigned)__popc(grp));
+                if (tok < n_cand) {
+                    srow[tok] = L;
+                    atomicAdd(&hist[dec::score_bin(__float_as_uint(L), base) * 32 + lane], 1u);
+                }
             }
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 256; i += blockDim.x)
-        if (hist[i]) atomicAdd(hist_g + b * 256 + i, hist[i]);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) {
+        unsigned c = 0;
+        for (int l = 0; l < 32; l++) c += hist[i * 32 + ((l + i) & 31)];  // banks differ
+        if (c) atomicAdd(hist_g + b * 256 + i, c);
+    }
 }
 
 struct GatherShared {
@@ -179,15 +182,27 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
         const float eps = (float)Hq * 0x1p-23f;
         const float thr = (E - eps) * (8.f / 9.f) * (1.f - 0x1p-10f);
         const float* srow = lrow + (size_t)b * score_ld;
-        // chunks start on 128-token boundaries; score rows are padded to 4
-        for (int s0 = s_begin + 4 * (int)threadIdx.x; s0 < s_end; s0 += 4 * kGatherThreads) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(srow + s0));
-            const float e[4] = {v.x, v.y, v.z, v.w};
+        // chunks start on 128-token boundaries; score rows are padded to 4;
+        // eight 16-byte loads in flight per thread
+        constexpr int U = 8;
+        for (int s0 = s_begin + 4 * (int)threadIdx.x; s0 < s_end; s0 += 4 * U * kGatherThreads) {
+            float4 v[U];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                if (s0 + i < s_end && e[i] >= thr) {
-                    const unsigned p = atomicAdd(&sh.n_cand, 1u);
-                    if (p < (unsigned)kCandCap) sh.cand[p] = s0 + i;
+            for (int u = 0; u < U; u++) {
+                const int s = s0 + u * 4 * kGatherThreads;
+                v[u] = s < s_end ? __ldcg(reinterpret_cast<const float4*>(srow + s))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    const int s = s0 + u * 4 * kGatherThreads + i;
+                    if (s < s_end && e[i] >= thr) {
+                        const unsigned p = atomicAdd(&sh.n_cand, 1u);
+                        if (p < (unsigned)kCandCap) sh.cand[p] = s;
+                    }
                 }
             }
         }

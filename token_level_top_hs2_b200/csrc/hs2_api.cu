@@ -12,6 +12,7 @@
 #include "../../include/hs2.h"
 #include "decode_kernels.cuh"
 #include "decode_stream.cuh"
+#include "decode_pass1.cuh"
 #include "decode_sketch.cuh"
 #include "decode_tc.cuh"
 #include "prefill_kernels.cuh"
@@ -377,13 +378,13 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     if constexpr (FP8 && D == 128) {
         // tensor-memory path: tokens as the MMA M dimension, exact f16 K/V
         const float qk2 = s->scale * kLog2e;
-        using LY = dtc::Layout<true>;
-        using LY2 = dtc::Layout<false>;
+        using LY = dtc::P1Layout;
+        using LY2 = dtc::Layout;
         const bool sketch = decode_uses_sketch(s);
         uint8_t* skt = sketch ? ws + w.sketch_off : nullptr;
         float* rsnap = reinterpret_cast<float*>(ws + w.rsnap_off);
         if (!set_smem(dtc::pass1_tc_kernel, LY::SMEM)) return HS2_ERR_CUDA;
-        dtc::pass1_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kThreads, LY::SMEM, st>>>(
+        dtc::pass1_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kP1Threads, LY::SMEM, st>>>(
             mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len, w.n_chunks, qk2, part,
             cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), skt, rsnap, w.sk_tiles, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
