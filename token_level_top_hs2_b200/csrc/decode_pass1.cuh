@@ -10,18 +10,20 @@
 // Per 128-token tile, with the tokens as the MMA M dimension:
 //   S^T[token][head] = K_tile (128 x 128, f16, TMEM) * Q^T (128 x 16, f16)
 //   O^T[dim][head]  += V_tile^T (128 x 128, f16, smem) * P (128 x 16, f16)
-// Roles (12 warps):
+// Roles (19 warps):
 //   warp 0       TMA producer: raw e4m3 K, V tiles and both scale rows into a
 //                ring of kNR stages;
-//   warp 1       MMA issuer: a non-blocking scheduler that issues whichever of
-//                QK(next) / PV(next) has its operands ready, so a tile's QK
-//                never waits behind an older tile's PV;
-//   warps 2-5    K converters: thread = token row = TMEM lane; e4m3 -> f16
+//   warp 1       QK issuer (one thread); TMEM owner;
+//   warp 2       PV issuer (one thread): a single thread issues one tcgen05.mma
+//                per ~130 cycles whatever its N, so the 16 N=16 MMAs of a tile
+//                are spread over two issuers;
+//   warps 3-6    K converters: thread = token row = TMEM lane; e4m3 -> f16
 //                straight into one of kDK TMEM K buffers; copy both scales;
-//   warps 6-9    softmax: thread = token = TMEM lane of S^T; lazily raised
-//                CTA-wide running max; P (f16, K-major) into one of kDV shared
-//                buffers; the per-token sketch bytes;
-//   warps 10-11  V converters: two token rows per thread, e4m3 -> f16 into one
+//   warps 7-14   softmax, two groups of 4 warps owning heads 0-7 and 8-15:
+//                thread = token = TMEM lane of S^T; per group, lazily raised
+//                running maxima shared by its 128 threads; P (f16, K-major)
+//                into one of kDP shared buffers; the per-token sketch bytes;
+//   warps 15-18  V converters: one token row per thread, e4m3 -> f16 into one
 //                of kDV shared V tiles (canonical 128-byte-swizzled layout).
 // K and V conversion run in separate warps so that the QK/softmax chain of
 // later tiles proceeds while an older tile's PV is still pending.
@@ -32,10 +34,17 @@
 namespace hs2 {
 namespace dtc {
 
-constexpr int kP1Threads = 384;
+// warp roles
+constexpr int kWProd = 0, kWQK = 1, kWPV = 2;
+constexpr int kWK0 = 3;                 // 4 K-converter warps: lane quarters 3, 0, 1, 2
+constexpr int kWS0 = kWK0 + 4;          // 2 x 4 softmax warps (heads 0-7, 8-15)
+constexpr int kWV0 = kWS0 + 8;          // V-converter warps
+constexpr int kVW = 4;                  // V-converter warps (128 / (32 kVW) rows each)
+constexpr int kP1Threads = 32 * (kWV0 + kVW);
 constexpr int kNR = 4;  // raw stages
 constexpr int kDK = 4;  // K tiles in TMEM = S^T buffers = scale slots
-constexpr int kDV = 2;  // f16 V tiles and P tiles in shared memory
+constexpr int kDV = 2;  // f16 V tiles in shared memory
+constexpr int kDP = 4;  // P tiles in shared memory
 // TMEM columns (512 allocated, one CTA per SM): S^T buffers, O^T, K tiles
 constexpr uint32_t P1_COL_S = 0, P1_COL_O = 16 * kDK, P1_COL_K = 128;
 static_assert(P1_COL_O + 16 <= P1_COL_K && P1_COL_K + 64 * kDK <= 512, "TMEM plan");
@@ -50,8 +59,8 @@ struct P1Layout {
     static constexpr int OFF_VF = OFF_RAW + kNR * RAW;
     static constexpr int OFF_QF = OFF_VF + kDV * F16T;
     static constexpr int OFF_P = OFF_QF + PT;
-    static constexpr int OFF_SC = OFF_P + kDV * PT;        // sk[kDK][128], sv[kDK][128]
-    static constexpr int OFF_RED = OFF_SC + 2 * kDK * TOK * 4;  // [4][16] floats
+    static constexpr int OFF_SC = OFF_P + kDP * PT;        // sk[kDK][128], sv[kDK][128]
+    static constexpr int OFF_RED = OFF_SC + 2 * kDK * TOK * 4;  // [2][4][8] floats
     static constexpr int SMEM = OFF_RED + 4 * 16 * 4 + 1024;
     static_assert(RAW >= RAW_SV + TOK * 4 && RAW % 1024 == 0, "raw stage");
     static_assert(OFF_VF % 1024 == 0 && OFF_QF % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
@@ -61,30 +70,10 @@ struct P1Layout {
 struct P1Bars {
     uint64_t raw_full[kNR], raw_empty[kNR];
     uint64_t q_ready, kf_full[kDK], kf_empty[kDK], s_full[kDK], s_empty[kDK];
-    uint64_t vf_full[kDV], vf_empty[kDV], p_full[kDV], p_empty[kDV], drain;
+    uint64_t vf_full[kDV], vf_empty[kDV], p_full[kDP], p_empty[kDP], drain_qk, drain_pv;
     uint32_t tmem_base;
     int abort_;
     unsigned last;
-};
-
-// Spin guard of the MMA scheduler: after kWaitNs without progress it raises
-// the abort flag (everybody's bounded waits then give up) and FLAG_TIMEOUT.
-struct SpinGuard {
-    uint64_t t0 = 0;
-    uint32_t i = 0;
-    HS2_DEV void progress() { i = 0; t0 = 0; }
-    HS2_DEV bool idle(volatile int* abort_, unsigned* flags) {
-        if ((++i & 255u) != 0) return true;
-        if (*abort_) return false;
-        const uint64_t now = globaltimer_ns();
-        if (t0 == 0) t0 = now;
-        if (now - t0 > kWaitNs) {
-            *abort_ = 1;
-            atomicOr(flags, FLAG_TIMEOUT);
-            return false;
-        }
-        return true;
-    }
 };
 
 HS2_DEV void p1_issue_raw(uint8_t* st, const CUtensorMap* mk, const CUtensorMap* mv,
@@ -132,26 +121,29 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNR; i++) {
             mbar_init(&bars.raw_full[i], 1);
-            mbar_init(&bars.raw_empty[i], 6);  // 4 K-converter + 2 V-converter warps
+            mbar_init(&bars.raw_empty[i], 4 + kVW);  // K- and V-converter warps
         }
         mbar_init(&bars.q_ready, 4);
         for (int i = 0; i < kDK; i++) {
             mbar_init(&bars.kf_full[i], 4);
             mbar_init(&bars.kf_empty[i], 1);
             mbar_init(&bars.s_full[i], 1);
-            mbar_init(&bars.s_empty[i], 4);
+            mbar_init(&bars.s_empty[i], 8);
         }
         for (int i = 0; i < kDV; i++) {
-            mbar_init(&bars.vf_full[i], 2);
+            mbar_init(&bars.vf_full[i], kVW);
             mbar_init(&bars.vf_empty[i], 1);
-            mbar_init(&bars.p_full[i], 4);
+        }
+        for (int i = 0; i < kDP; i++) {
+            mbar_init(&bars.p_full[i], 8);
             mbar_init(&bars.p_empty[i], 1);
         }
-        mbar_init(&bars.drain, 1);
+        mbar_init(&bars.drain_qk, 1);
+        mbar_init(&bars.drain_pv, 1);
         bars.abort_ = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kWQK) {
         tmem_alloc(&bars.tmem_base, 512);
         tmem_relinquish();
     }
@@ -160,7 +152,7 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     fence_after_sync();
     const uint32_t tmem = bars.tmem_base;
 
-    if (warp == 0) {
+    if (warp == kWProd) {
         if (lane == 0 && n > 0) {
             // ------------------------------------------------------ producer
             int armed = 0;
@@ -177,57 +169,55 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     mbar_wait(&bars.raw_full[j % kNR], (j / kNR) & 1, &no_abort, flags);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == kWQK) {
         if (lane == 0 && n > 0) {
-            // --------------------------------------------- MMA scheduler
+            // -------------------------------------------------- QK issuer
             constexpr uint32_t id_qk = idesc_f16(128, 16, false, false);
-            constexpr uint32_t id_pv = idesc_f16(128, 16, true, false);
-            const uint32_t vf = smem_u32(smem + LY::OFF_VF);
-            const uint32_t qf = smem_u32(smem + LY::OFF_QF), pf = smem_u32(smem + LY::OFF_P);
+            const uint32_t qf = smem_u32(smem + LY::OFF_QF);
             bool ok = mbar_wait(&bars.q_ready, 0, abort_, flags);
-            int nq = 0, np = 0;  // next QK / PV tile
-            SpinGuard guard;
-            while (ok && np < n) {
-                const int vb = np % kDV, vu = np / kDV;
-                if (np < nq && mbar_try_wait(&bars.p_full[vb], vu & 1) &&
-                    mbar_try_wait(&bars.vf_full[vb], vu & 1)) {
-                    fence_after_sync();
+            for (int j = 0; ok && j < n; j++) {
+                const int kb = j % kDK, ku = j / kDK;
+                if (!mbar_wait(&bars.kf_full[kb], ku & 1, abort_, flags)) break;
+                if (ku > 0 && !mbar_wait(&bars.s_empty[kb], (ku - 1) & 1, abort_, flags)) break;
+                fence_after_sync();
 #pragma unroll
-                    for (int ks = 0; ks < 8; ks++) {
-                        const uint32_t va = vf + vb * LY::F16T + ks * (16 * 128);
-                        const uint32_t pb = pf + vb * LY::PT + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
-                        mma_ss(tmem + P1_COL_O, sdesc_sw128(va, TOK * 128, 1024),
-                               sdesc_sw128(pb, 16, 1024), id_pv, (np > 0 || ks > 0) ? 1u : 0u);
-                    }
-                    mma_commit(&bars.vf_empty[vb]);
-                    mma_commit(&bars.p_empty[vb]);
-                    np++;
-                    guard.progress();
-                    continue;
+                for (int ks = 0; ks < 8; ks++) {
+                    const uint32_t kbq = qf + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
+                    mma_ts(tmem + P1_COL_S + kb * 16, tmem + P1_COL_K + kb * 64 + ks * 8,
+                           sdesc_sw128(kbq, 16, 1024), id_qk, ks > 0);
                 }
-                const int kb = nq % kDK, ku = nq / kDK;
-                if (nq < n && mbar_try_wait(&bars.kf_full[kb], ku & 1) &&
-                    (ku == 0 || mbar_try_wait(&bars.s_empty[kb], (ku - 1) & 1))) {
-                    fence_after_sync();
-#pragma unroll
-                    for (int ks = 0; ks < 8; ks++) {
-                        const uint32_t kbq = qf + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
-                        mma_ts(tmem + P1_COL_S + kb * 16, tmem + P1_COL_K + kb * 64 + ks * 8,
-                               sdesc_sw128(kbq, 16, 1024), id_qk, ks > 0);
-                    }
-                    mma_commit(&bars.s_full[kb]);
-                    mma_commit(&bars.kf_empty[kb]);
-                    nq++;
-                    guard.progress();
-                    continue;
-                }
-                ok = guard.idle(abort_, flags);
+                mma_commit(&bars.s_full[kb]);
+                mma_commit(&bars.kf_empty[kb]);
             }
-            mma_commit(&bars.drain);
+            mma_commit(&bars.drain_qk);
             volatile int no_abort = 0;
-            mbar_wait(&bars.drain, 0, &no_abort, flags);
+            mbar_wait(&bars.drain_qk, 0, &no_abort, flags);
         }
-    } else if (warp < 6) {
+    } else if (warp == kWPV) {
+        if (lane == 0 && n > 0) {
+            // -------------------------------------------------- PV issuer
+            constexpr uint32_t id_pv = idesc_f16(128, 16, true, false);
+            const uint32_t vf = smem_u32(smem + LY::OFF_VF), pf = smem_u32(smem + LY::OFF_P);
+            for (int j = 0; j < n; j++) {
+                const int vb = j % kDV, vu = j / kDV, pbf = j % kDP, pu = j / kDP;
+                if (!mbar_wait(&bars.p_full[pbf], pu & 1, abort_, flags)) break;
+                if (!mbar_wait(&bars.vf_full[vb], vu & 1, abort_, flags)) break;
+                fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 8; ks++) {
+                    const uint32_t va = vf + vb * LY::F16T + ks * (16 * 128);
+                    const uint32_t pb = pf + pbf * LY::PT + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
+                    mma_ss(tmem + P1_COL_O, sdesc_sw128(va, TOK * 128, 1024),
+                           sdesc_sw128(pb, 16, 1024), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
+                }
+                mma_commit(&bars.vf_empty[vb]);
+                mma_commit(&bars.p_empty[pbf]);
+            }
+            mma_commit(&bars.drain_pv);
+            volatile int no_abort = 0;
+            mbar_wait(&bars.drain_pv, 0, &no_abort, flags);
+        }
+    } else if (warp < kWS0) {
         // ---------------------------------------------------- K converters
         const int t = (warp & 3) * 32 + lane;  // token row = TMEM lane of this warp
         const uint32_t k_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16) + P1_COL_K;
@@ -263,9 +253,9 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             }
         }
         if (__any_sync(0xffffffffu, bad_scale) && lane == 0) atomicOr(flags, FLAG_SCALE_RANGE);
-    } else if (warp >= 10) {
+    } else if (warp >= kWV0) {
         // ---------------------------------------------------- V converters
-        const int v = (warp - 10) * 32 + lane;  // rows v and v + 64
+        const int v = (warp - kWV0) * 32 + lane;  // rows v, v + 32 kVW, ...
         for (int j = 0; j < n; j++) {
             const int st = j % kNR, vb = j % kDV, vu = j / kDV;
             if (!mbar_wait(&bars.raw_full[st], (j / kNR) & 1, abort_, flags)) break;
@@ -273,8 +263,8 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             const uint8_t* raw = smem + LY::OFF_RAW + st * LY::RAW + LY::RAW_V;
             uint8_t* dst = smem + LY::OFF_VF + vb * LY::F16T;
             const int row0 = s_begin + j * TOK;
-            convert_row(raw, dst, v, row0 + v < s_end);
-            convert_row(raw, dst, v + 64, row0 + v + 64 < s_end);
+#pragma unroll
+            for (int r = v; r < TOK; r += 32 * kVW) convert_row(raw, dst, r, row0 + r < s_end);
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) {
@@ -284,28 +274,35 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         }
     } else {
         // ----------------------------------------------------------- softmax
+        // group g owns heads 8g .. 8g+7 for all 128 tokens of a tile: its own
+        // running references, partial sums, votes and O^T columns
+        constexpr int NH = 8;
+        const int g = (warp - kWS0) >> 2;
+        const int h0 = NH * g;
         const int wq = warp & 3;                 // TMEM lane quarter of this warp
         const int t = wq * 32 + lane;            // token row = TMEM lane
         const uint32_t lane_addr = tmem + ((uint32_t)(wq * 32) << 16);
+        float* gred = red + g * (4 * NH);        // [4][NH]
+        const int bar_vote = 1 + 2 * g, bar_red = 2 + 2 * g;
         uint8_t* pf = smem + LY::OFF_P;
         // R = running max - kSk: probabilities are formed as 2^(x - R), in
         // (0, 2^(kLazy + kSk)], which is the range the sketch codes cover
-        float R[16], l[16];
+        float R[NH], l[NH];
 #pragma unroll
-        for (int h = 0; h < 16; h++) {
+        for (int h = 0; h < NH; h++) {
             R[h] = -INFINITY;
             l[h] = 0.f;
         }
         bool ok = true;
         for (int j = 0; j < n; j++) {
-            const int kb = j % kDK, vb = j % kDV, vu = j / kDV;
+            const int kb = j % kDK, pbf = j % kDP, pu = j / kDP;
             if (!mbar_wait(&bars.s_full[kb], (j / kDK) & 1, abort_, flags)) {
                 ok = false;
                 break;
             }
             fence_after_sync();
-            uint32_t r[16];
-            tmem_ld16(lane_addr + P1_COL_S + kb * 16, r);
+            uint32_t r[NH];
+            tmem_ld8(lane_addr + P1_COL_S + kb * 16 + h0, r);
             tmem_ld_wait();
             const float ks = skb[kb * TOK + t] * qk_scale;
             const float sv = svb[kb * TOK + t] * (1.f / 64.f);
@@ -313,147 +310,147 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars.s_empty[kb]);
             const bool valid = s_begin + j * TOK + t < s_end;
-            float x[16];
+            float x[NH];
             bool over = false;
 #pragma unroll
-            for (int h = 0; h < 16; h++) {
+            for (int h = 0; h < NH; h++) {
                 x[h] = valid ? __uint_as_float(r[h]) * ks : -INFINITY;
                 over |= x[h] > R[h] + (kLazy + kSk);
             }
-            if (bar_red_or(over, 1, 128)) {
-                // raise the per-head running max to this tile's max
-                float mx[16];
+            if (bar_red_or(over, bar_vote, 128)) {
+                // raise this group's running maxima to the tile's maxima
+                float mx[NH];
 #pragma unroll
-                for (int h = 0; h < 16; h++) {
+                for (int h = 0; h < NH; h++) {
                     float v = x[h];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
                     mx[h] = v;
                 }
-                if (lane < 16) {
+                if (lane < NH) {
                     float v = mx[0];
 #pragma unroll
-                    for (int h = 1; h < 16; h++)
+                    for (int h = 1; h < NH; h++)
                         if (lane == h) v = mx[h];
-                    red[wq * 16 + lane] = v;
+                    gred[wq * NH + lane] = v;
                 }
-                bar_named(2, 128);
-                float alpha[16];
+                bar_named(bar_red, 128);
+                float alpha[NH];
                 bool any_scale = false;
 #pragma unroll
-                for (int h = 0; h < 16; h++) {
-                    const float tm = fmaxf(fmaxf(red[h], red[16 + h]), fmaxf(red[32 + h], red[48 + h]));
+                for (int h = 0; h < NH; h++) {
+                    const float tm = fmaxf(fmaxf(gred[h], gred[NH + h]),
+                                           fmaxf(gred[2 * NH + h], gred[3 * NH + h]));
                     const float nm = fmaxf(R[h], tm - kSk);
                     alpha[h] = (R[h] == -INFINITY || nm == R[h]) ? 1.f : ex2(R[h] - nm);
                     any_scale |= alpha[h] != 1.f;
                     R[h] = nm;
                     l[h] *= alpha[h];
                 }
-                bar_named(2, 128);  // red[] is read by everyone before it is reused
+                bar_named(bar_red, 128);  // gred[] is read by everyone before it is reused
                 if (j > 0 && any_scale) {
-                    // O^T holds tiles 0..j-1: wait for PV(j-1), scale its columns
-                    const int pb = (j - 1) % kDV, pu = (j - 1) / kDV;
-                    if (!mbar_wait(&bars.p_empty[pb], pu & 1, abort_, flags)) {
+                    // O^T holds tiles 0..j-1: wait for PV(j-1), scale this group's columns
+                    const int pb1 = (j - 1) % kDP, pu1 = (j - 1) / kDP;
+                    if (!mbar_wait(&bars.p_empty[pb1], pu1 & 1, abort_, flags)) {
                         ok = false;
                         break;
                     }
                     fence_after_sync();
-                    uint32_t o[16];
-                    tmem_ld16(lane_addr + P1_COL_O, o);
+                    uint32_t o[NH];
+                    tmem_ld8(lane_addr + P1_COL_O + h0, o);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int h = 0; h < 16; h++) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
-                    tmem_st16(lane_addr + P1_COL_O, o);
+                    for (int h = 0; h < NH; h++) o[h] = __float_as_uint(__uint_as_float(o[h]) * alpha[h]);
+                    tmem_st8(lane_addr + P1_COL_O + h0, o);
                     tmem_st_wait();
                     fence_before_sync();
                 }
             }
-            uint32_t pw[16];
-            float pr[16];
+            float pr[NH];
+            uint32_t pw[NH / 2];
 #pragma unroll
-            for (int h = 0; h < 16; h++) {
+            for (int h = 0; h < NH; h++) {
                 pr[h] = (valid && R[h] != -INFINITY) ? ex2(x[h] - R[h]) : 0.f;
                 l[h] += pr[h];
-                pw[h] = __half_as_ushort(__float2half_rn(pr[h] * sv));
             }
+#pragma unroll
+            for (int i = 0; i < NH / 2; i++) pw[i] = pack_f16(pr[2 * i] * sv, pr[2 * i + 1] * sv);
             if (sketch != nullptr) {
                 const int tok = s_begin + j * TOK + t;
                 if (valid) {
-                    uint32_t hw[8];
+                    uint32_t hw[NH / 2];
 #pragma unroll
-                    for (int i = 0; i < 8; i++) hw[i] = f16x2_rz(pr[2 * i], pr[2 * i + 1]);
-                    uint4 cw;
-                    cw.x = prmt(hw[0] >> 7, hw[1] >> 7, 0x6420u);
-                    cw.y = prmt(hw[2] >> 7, hw[3] >> 7, 0x6420u);
-                    cw.z = prmt(hw[4] >> 7, hw[5] >> 7, 0x6420u);
-                    cw.w = prmt(hw[6] >> 7, hw[7] >> 7, 0x6420u);
-                    *reinterpret_cast<uint4*>(sketch + ((size_t)b * Tmax + tok) * 16) = cw;
+                    for (int i = 0; i < NH / 2; i++) hw[i] = f16x2_rz(pr[2 * i], pr[2 * i + 1]);
+                    const uint2 cw = make_uint2(prmt(hw[0] >> 7, hw[1] >> 7, 0x6420u),
+                                                prmt(hw[2] >> 7, hw[3] >> 7, 0x6420u));
+                    *reinterpret_cast<uint2*>(sketch + ((size_t)b * Tmax + tok) * 16 + h0) = cw;
                 }
-                if (wq == 0 && lane < 16) {
+                if (wq == 0 && lane < NH) {
                     float rv = R[0];
 #pragma unroll
-                    for (int h = 1; h < 16; h++)
+                    for (int h = 1; h < NH; h++)
                         if (lane == h) rv = R[h];
-                    rsnap[((size_t)b * sk_tiles + (s_begin / TOK + j)) * 16 + lane] = rv;
+                    rsnap[((size_t)b * sk_tiles + (s_begin / TOK + j)) * 16 + h0 + lane] = rv;
                 }
             }
-            if (vu > 0 && !mbar_wait(&bars.p_empty[vb], (vu - 1) & 1, abort_, flags)) {
+            if (pu > 0 && !mbar_wait(&bars.p_empty[pbf], (pu - 1) & 1, abort_, flags)) {
                 ok = false;
                 break;
             }
-            uint8_t* pt = pf + vb * LY::PT;
+            uint8_t* pt = pf + pbf * LY::PT;
 #pragma unroll
-            for (int h = 0; h < 16; h++)
-                *reinterpret_cast<uint16_t*>(pt + f16_off(16, h, t)) = (uint16_t)pw[h];
+            for (int h = 0; h < NH; h++)
+                *reinterpret_cast<uint16_t*>(pt + f16_off(16, h0 + h, t)) =
+                    (uint16_t)(pw[h >> 1] >> (16 * (h & 1)));
             fence_proxy_async();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars.p_full[vb]);
+            if (lane == 0) mbar_arrive(&bars.p_full[pbf]);
         }
         // chunk partial: l summed over the tile rows, O^T from TMEM (lane = dim)
 #pragma unroll
-        for (int h = 0; h < 16; h++) {
+        for (int h = 0; h < NH; h++) {
             float v = l[h];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
             l[h] = v;
         }
-        if (lane < 16) {
+        if (lane < NH) {
             float v = l[0];
 #pragma unroll
-            for (int h = 1; h < 16; h++)
+            for (int h = 1; h < NH; h++)
                 if (lane == h) v = l[h];
-            red[wq * 16 + lane] = v;
+            gred[wq * NH + lane] = v;
         }
-        bar_named(2, 128);
+        bar_named(bar_red, 128);
         float* dst = part + ((size_t)b * n_chunks + chunk) * PART;
-        if (t < 16) {
+        if (t < NH) {
             float mt = R[0];
 #pragma unroll
-            for (int h = 1; h < 16; h++)
+            for (int h = 1; h < NH; h++)
                 if (t == h) mt = R[h];
             // O is relative to R + kSk (the P tiles carry sv / 64), so is the sum
-            dst[16 * D + t] = mt + kSk;
-            dst[16 * D + 16 + t] =
-                (red[t] + red[16 + t] + red[32 + t] + red[48 + t]) * (1.f / 64.f);
+            dst[16 * D + h0 + t] = mt + kSk;
+            dst[16 * D + 16 + h0 + t] =
+                (gred[t] + gred[NH + t] + gred[2 * NH + t] + gred[3 * NH + t]) * (1.f / 64.f);
         }
         // the last PV (and with it every earlier one) has completed once its
         // P buffer is released
         if (ok && n > 0 &&
-            mbar_wait(&bars.p_empty[(n - 1) % kDV], ((n - 1) / kDV) & 1, abort_, flags)) {
+            mbar_wait(&bars.p_empty[(n - 1) % kDP], ((n - 1) / kDP) & 1, abort_, flags)) {
             fence_after_sync();
-            uint32_t o[16];
-            tmem_ld16(lane_addr + P1_COL_O, o);
+            uint32_t o[NH];
+            tmem_ld8(lane_addr + P1_COL_O + h0, o);
             tmem_ld_wait();
 #pragma unroll
-            for (int h = 0; h < 16; h++) dst[h * D + t] = __uint_as_float(o[h]);
+            for (int h = 0; h < NH; h++) dst[(h0 + h) * D + t] = __uint_as_float(o[h]);
         } else {
 #pragma unroll
-            for (int h = 0; h < 16; h++) dst[h * D + t] = 0.f;
+            for (int h = 0; h < NH; h++) dst[(h0 + h) * D + t] = 0.f;
         }
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWQK) {
         fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
