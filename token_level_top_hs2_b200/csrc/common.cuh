@@ -70,6 +70,15 @@ HS2_DEV uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
+// Transposing load of a 16 x 16 byte block (threads 0..15 give the 16 row
+// addresses, 16-byte aligned): thread L receives column L/4 (r0) and column
+// L/4 + 8 (r1), rows 4(L%4) .. 4(L%4)+3 in bytes 0..3 of each.
+HS2_DEV void ldmatrix_t16_b8(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x1.trans.shared.b8 {%0, %1}, [%2];"
+                 : "=r"(r0), "=r"(r1)
+                 : "r"(addr));
+}
+
 // Two floats -> f16x2 rounded toward zero: lo in bits 0..15, hi in bits 16..31.
 HS2_DEV uint32_t f16x2_rz(float lo, float hi) {
     uint32_t r;

@@ -9,7 +9,7 @@
 //
 // Per 128-token tile, with the tokens as the MMA M dimension:
 //   S^T[token][head] = K_tile (128 x 128, f16, TMEM) * Q^T (128 x 16, f16)
-//   O^T[dim][head]  += V_tile^T (128 x 128, f16, smem) * P (128 x 16, f16)
+//   O^T[dim][head]  += V_tile^T (128 x 128, f16, TMEM) * P (128 x 16, f16)
 // Roles (19 warps):
 //   warp 0       TMA producer: raw e4m3 K, V tiles and both scale rows into a
 //                ring of kNR stages;
@@ -23,8 +23,9 @@
 //                thread = token = TMEM lane of S^T; per group, lazily raised
 //                running maxima shared by its 128 threads; P (f16, K-major)
 //                into one of kDP shared buffers; the per-token sketch bytes;
-//   warps 15-18  V converters: one token row per thread, e4m3 -> f16 into one
-//                of kDV shared V tiles (canonical 128-byte-swizzled layout).
+//   warps 15-18  V converters: e4m3 -> f16 V^T straight into one of kDV TMEM
+//                tiles (lane = dim), the A operand of PV, through transposing
+//                16 x 16 byte shared-memory loads.
 // K and V conversion run in separate warps so that the QK/softmax chain of
 // later tiles proceeds while an older tile's PV is still pending.
 #pragma once
@@ -39,31 +40,31 @@ constexpr int kWProd = 0, kWQK = 1, kWPV = 2;
 constexpr int kWK0 = 3;                 // 4 K-converter warps: lane quarters 3, 0, 1, 2
 constexpr int kWS0 = kWK0 + 4;          // 2 x 4 softmax warps (heads 0-7, 8-15)
 constexpr int kWV0 = kWS0 + 8;          // V-converter warps
-constexpr int kVW = 4;                  // V-converter warps (128 / (32 kVW) rows each)
+constexpr int kVW = 4;                  // V-converter warps, one per TMEM lane quarter
 constexpr int kP1Threads = 32 * (kWV0 + kVW);
-constexpr int kNR = 4;  // raw stages
+constexpr int kNR = 5;  // raw stages
 constexpr int kDK = 4;  // K tiles in TMEM = S^T buffers = scale slots
-constexpr int kDV = 2;  // f16 V tiles in shared memory
+constexpr int kDV = 2;  // f16 V^T tiles in TMEM
 constexpr int kDP = 4;  // P tiles in shared memory
 // TMEM columns (512 allocated, one CTA per SM): S^T buffers, O^T, K tiles
-constexpr uint32_t P1_COL_S = 0, P1_COL_O = 16 * kDK, P1_COL_K = 128;
-static_assert(P1_COL_O + 16 <= P1_COL_K && P1_COL_K + 64 * kDK <= 512, "TMEM plan");
+// TMEM columns: S^T buffers, O^T, K tiles (lane = token), V^T tiles (lane = dim)
+constexpr uint32_t P1_COL_S = 0, P1_COL_O = 16 * kDK, P1_COL_K = 128,
+                   P1_COL_V = P1_COL_K + 64 * kDK;
+static_assert(P1_COL_O + 16 <= P1_COL_K && P1_COL_V + 64 * kDV <= 512, "TMEM plan");
 
 struct P1Layout {
     static constexpr int RAW_K = 0, RAW_V = TOK * 128;
     static constexpr int RAW_SK = 2 * TOK * 128, RAW_SV = RAW_SK + TOK * 4;
     static constexpr int RAW = 34816;                      // stage stride, 1024-aligned
-    static constexpr int F16T = 2 * TOK * 128;             // f16 V tile
     static constexpr int PT = 2 * 16 * 128;                // P tile: 2 blocks of 16 x 128 B
     static constexpr int OFF_RAW = 0;
-    static constexpr int OFF_VF = OFF_RAW + kNR * RAW;
-    static constexpr int OFF_QF = OFF_VF + kDV * F16T;
+    static constexpr int OFF_QF = OFF_RAW + kNR * RAW;
     static constexpr int OFF_P = OFF_QF + PT;
     static constexpr int OFF_SC = OFF_P + kDP * PT;        // sk[kDK][128], sv[kDK][128]
     static constexpr int OFF_RED = OFF_SC + 2 * kDK * TOK * 4;  // [2][4][8] floats
     static constexpr int SMEM = OFF_RED + 4 * 16 * 4 + 1024;
     static_assert(RAW >= RAW_SV + TOK * 4 && RAW % 1024 == 0, "raw stage");
-    static_assert(OFF_VF % 1024 == 0 && OFF_QF % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
+    static_assert(OFF_QF % 1024 == 0 && OFF_P % 1024 == 0, "alignment");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
@@ -196,8 +197,8 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     } else if (warp == kWPV) {
         if (lane == 0 && n > 0) {
             // -------------------------------------------------- PV issuer
-            constexpr uint32_t id_pv = idesc_f16(128, 16, true, false);
-            const uint32_t vf = smem_u32(smem + LY::OFF_VF), pf = smem_u32(smem + LY::OFF_P);
+            constexpr uint32_t id_pv = idesc_f16(128, 16, false, false);
+            const uint32_t pf = smem_u32(smem + LY::OFF_P);
             for (int j = 0; j < n; j++) {
                 const int vb = j % kDV, vu = j / kDV, pbf = j % kDP, pu = j / kDP;
                 if (!mbar_wait(&bars.p_full[pbf], pu & 1, abort_, flags)) break;
@@ -205,9 +206,8 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < 8; ks++) {
-                    const uint32_t va = vf + vb * LY::F16T + ks * (16 * 128);
                     const uint32_t pb = pf + pbf * LY::PT + (ks >> 2) * (16 * 128) + (ks & 3) * 32;
-                    mma_ss(tmem + P1_COL_O, sdesc_sw128(va, TOK * 128, 1024),
+                    mma_ts(tmem + P1_COL_O, tmem + P1_COL_V + vb * 64 + ks * 8,
                            sdesc_sw128(pb, 16, 1024), id_pv, (j > 0 || ks > 0) ? 1u : 0u);
                 }
                 mma_commit(&bars.vf_empty[vb]);
@@ -255,17 +255,44 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         if (__any_sync(0xffffffffu, bad_scale) && lane == 0) atomicOr(flags, FLAG_SCALE_RANGE);
     } else if (warp >= kWV0) {
         // ---------------------------------------------------- V converters
-        const int v = (warp - kWV0) * 32 + lane;  // rows v, v + 32 kVW, ...
+        // V^T into TMEM, lane = dim: this warp owns dims 32 q4 .. 32 q4 + 31.
+        // A transposing 16 x 16 byte load gives thread (g = lane/4, tq = lane%4)
+        // dims g and g + 8 of a 16-dim block, tokens 4 tq .. 4 tq + 3 of a
+        // 16-token block; converted, they are exactly what a 16x256b TMEM
+        // store puts in lanes g, g + 8 and columns 2 tq, 2 tq + 1 (column c
+        // holds tokens 2c, 2c + 1).
+        const int q4 = warp & 3;
+        const int tq = lane & 3;
+        const uint32_t v_base = tmem + ((uint32_t)(q4 * 32) << 16) + P1_COL_V;
         for (int j = 0; j < n; j++) {
             const int st = j % kNR, vb = j % kDV, vu = j / kDV;
             if (!mbar_wait(&bars.raw_full[st], (j / kNR) & 1, abort_, flags)) break;
             if (vu > 0 && !mbar_wait(&bars.vf_empty[vb], (vu - 1) & 1, abort_, flags)) break;
+            fence_after_sync();
             const uint8_t* raw = smem + LY::OFF_RAW + st * LY::RAW + LY::RAW_V;
-            uint8_t* dst = smem + LY::OFF_VF + vb * LY::F16T;
             const int row0 = s_begin + j * TOK;
 #pragma unroll
-            for (int r = v; r < TOK; r += 32 * kVW) convert_row(raw, dst, r, row0 + r < s_end);
-            fence_proxy_async();
+            for (int h = 0; h < 2; h++) {
+                const int c = 2 * q4 + h;  // 16-byte chunk = dims 16c .. 16c + 15
+#pragma unroll
+                for (int kb = 0; kb < 8; kb++) {
+                    const int r = kb * 16 + (lane & 15);
+                    uint32_t b0, b1;
+                    ldmatrix_t16_b8(smem_u32(raw + r * 128 + ((c ^ (r & 7)) << 4)), b0, b1);
+                    // tokens past the chunk end (e.g. beyond the length) become zeros
+                    const int nv = s_end - (row0 + kb * 16 + 4 * tq);
+                    if (nv < 4) {
+                        const uint32_t m = nv <= 0 ? 0u : (1u << (8 * nv)) - 1u;
+                        b0 &= m;
+                        b1 &= m;
+                    }
+                    tmem_st_16x256b(v_base + ((uint32_t)(16 * h) << 16) + vb * 64 + kb * 8,
+                                    e4m3x2_lo_to_f16x2(b0), e4m3x2_lo_to_f16x2(b0 >> 16),
+                                    e4m3x2_lo_to_f16x2(b1), e4m3x2_lo_to_f16x2(b1 >> 16));
+                }
+            }
+            tmem_st_wait();
+            fence_before_sync();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bars.vf_full[vb]);

@@ -189,6 +189,14 @@ HS2_DEV void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
                  "r"(r[7])
                  : "memory");
 }
+// 16 lanes x 256 bits: thread T writes lane base + T/4 (r0, r1 into columns
+// 2(T%4), 2(T%4)+1) and lane base + T/4 + 8 (r2, r3 into the same columns) --
+// the layout of an mma accumulator fragment.
+HS2_DEV void tmem_st_16x256b(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x1.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+                 : "memory");
+}
 HS2_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ------------------------------------------------------------- descriptors
