@@ -22,8 +22,10 @@
 // sketch_gather_kernel  the bin holding the k-th largest L gives E, a lower
 //                       bound of the k-th largest score.  A token can be in
 //                       the top k only if 9/8 L + eps >= E; exactly those are
-//                       rescored from their K rows (a thread per token) and
-//                       the exact top k is cut from them.
+//                       rescored from their K rows (a thread per token); the
+//                       last CTA of the sequence bins their exact scores, takes
+//                       every key above the bin of the k-th and ranks the
+//                       keys inside that bin (ties to the lower position).
 // If a sequence's candidates overflow the boundary buffer (many near-equal
 // scores, e.g. repeated keys), it is flagged and the exact pass 2 and its
 // gather run for that sequence instead (their launches are gated on the flag).
@@ -36,7 +38,7 @@ namespace dsk {
 
 constexpr int TOK = 128;
 constexpr int kScoreThreads = 256;
-constexpr int kGatherThreads = 256;
+constexpr int kGatherThreads = 512;
 constexpr int kCandCap = 2048;  // candidates one CTA may rescore
 
 // ----------------------------------------------------------------------------
@@ -123,8 +125,8 @@ struct GatherShared {
     float q[16][128];     // f16-rounded query, as the MMA operand saw it
     int cand[kCandCap];   // this CTA's candidate positions
     int hist[260];
-    int bin;
-    unsigned n_cand, last;
+    int bin, above;
+    unsigned n_cand, n_out, last;
 };
 
 // ----------------------------------------------------------------------------
@@ -139,8 +141,7 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
                      float qk2, const int32_t* __restrict__ lengths, int Tmax, int Hq, int W, int k,
                      int chunk_len, int n_chunks, unsigned* __restrict__ bnd_cnt,
                      uint64_t* __restrict__ bnd, unsigned* __restrict__ ovf,
-                     unsigned* __restrict__ counter, unsigned* __restrict__ out_cnt,
-                     int32_t* __restrict__ idx) {
+                     unsigned* __restrict__ counter, int32_t* __restrict__ idx) {
     extern __shared__ uint64_t skeys[];
     __shared__ GatherShared sh;
     const int b = blockIdx.y, chunk = blockIdx.x;
@@ -281,14 +282,61 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
             if (threadIdx.x == 0) atomicOr(ovf + b, 1u);
             return;
         }
+        // the exact top k of the candidates' keys: bin them by score, take
+        // every key above the bin of the k-th, rank the keys inside that bin
         const int nb = (int)nb_all;
-        for (int i = threadIdx.x; i < nb; i += blockDim.x)
-            skeys[i] = __ldcg(bnd + (size_t)b * dec::BCAP + i);
+        const uint32_t base = dec::seq_base(Hq, T);
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) sh.hist[i] = 0;
+        if (threadIdx.x == 0) {
+            sh.n_cand = 0;  // boundary keys gathered
+            sh.n_out = 0;   // keys written
+        }
         __syncthreads();
-        const uint64_t thr = block_radix_threshold([&](int i) { return skeys[i]; }, nb, k, sh.hist);
+        constexpr int PER = dec::BCAP / kGatherThreads;
+        uint64_t kv[PER];
+#pragma unroll
+        for (int u = 0; u < PER; u++) {
+            const int i = threadIdx.x + u * kGatherThreads;
+            kv[u] = i < nb ? __ldcg(bnd + (size_t)b * dec::BCAP + i) : 0ull;
+        }
+#pragma unroll
+        for (int u = 0; u < PER; u++) {
+            const int i = threadIdx.x + u * kGatherThreads;
+            const int bn = i < nb ? dec::score_bin((uint32_t)(kv[u] >> 32), base) : -1;
+            const unsigned grp = __match_any_sync(0xffffffffu, bn);
+            if (bn >= 0 && lane == __ffs(grp) - 1) atomicAdd(&sh.hist[bn], __popc(grp));
+        }
         __syncthreads();
-        for (int i = threadIdx.x; i < nb; i += blockDim.x)
-            if (skeys[i] >= thr) row[wl + atomicAdd(out_cnt + b, 1u)] = (int32_t)key_pos(skeys[i]);
+        if (warp == 0) {
+            int above, in_bin;
+            const int j = warp_find_bin(sh.hist, k, &above, &in_bin);
+            if (lane == 0) {
+                sh.bin = j;
+                sh.above = above;
+            }
+        }
+        __syncthreads();
+        const int jb = sh.bin, need = k - sh.above;
+        // keys above the boundary bin are in; the boundary bin's go to skeys
+#pragma unroll
+        for (int u = 0; u < PER; u++) {
+            const int i = threadIdx.x + u * kGatherThreads;
+            if (i >= nb) continue;
+            const int bn = dec::score_bin((uint32_t)(kv[u] >> 32), base);
+            if (bn > jb)
+                row[wl + atomicAdd(&sh.n_out, 1u)] = (int32_t)key_pos(kv[u]);
+            else if (bn == jb)
+                skeys[atomicAdd(&sh.n_cand, 1u)] = kv[u];
+        }
+        __syncthreads();
+        // keys are unique: the rank of a boundary key among its bin decides
+        const int m = (int)sh.n_cand;
+        for (int i = threadIdx.x; i < m; i += blockDim.x) {
+            const uint64_t key = skeys[i];
+            int rank = 0;
+            for (int q = 0; q < m; q++) rank += skeys[q] > key;
+            if (rank < need) row[wl + atomicAdd(&sh.n_out, 1u)] = (int32_t)key_pos(key);
+        }
     }
     for (int i = threadIdx.x; i < wl; i += blockDim.x) row[i] = t - wl + 1 + i;
     for (int i = wl + n_glob + threadIdx.x; i < S; i += blockDim.x) row[i] = -1;

@@ -314,7 +314,7 @@ DecodeWs2 decode_ws2(const hs2_decode_shape* s) {
     const size_t part_floats = (size_t)16 * s->d + 32;
     size_t off = 0;
     // zeroed per call: pass-1 counter, gather counter, out count, boundary count,
-    // histogram; then the sketch selection's counter, out count, boundary
+    // histogram; then the sketch selection's counter, (a spare word), boundary
     // count, overflow flag and histogram
     w.zero_off = off;
     w.zero_bytes = B * (8 + 512) * sizeof(unsigned);
@@ -353,7 +353,6 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     unsigned* bnd_cnt = zero + 3 * B;
     unsigned* hist = zero + 4 * B;
     unsigned* sk_cnt = zero + 260 * B;
-    unsigned* sk_out = zero + 261 * B;
     unsigned* sk_bnd = zero + 262 * B;
     unsigned* sk_ovf = zero + 263 * B;
     unsigned* sk_hist = zero + 264 * B;
@@ -400,7 +399,7 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
             dsk::sketch_gather_kernel<<<dim3(w.n_chunks, s->B), dsk::kGatherThreads, smem, st>>>(
                 scores, w.score_ld, sk_hist, static_cast<const uint8_t*>(kc), ks, qp, lse2, qk2,
                 lengths, s->Tmax, s->Hq, s->W, s->k, w.chunk_len, w.n_chunks, sk_bnd, bnd, sk_ovf,
-                sk_cnt, sk_out, idx);
+                sk_cnt, idx);
             if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
             // sequences whose candidates overflowed: exact scores, then the exact gather
             if (!set_smem(dtc::pass2_tc_kernel, LY2::SMEM)) return HS2_ERR_CUDA;
