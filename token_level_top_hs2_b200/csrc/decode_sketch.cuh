@@ -22,7 +22,7 @@
 // sketch_gather_kernel  the bin holding the k-th largest L gives E, a lower
 //                       bound of the k-th largest score.  A token can be in
 //                       the top k only if 9/8 L + eps >= E; exactly those are
-//                       rescored from their K rows (a thread per token); the
+//                       rescored from their K rows (a thread pair per token); the
 //                       last CTA of the sequence bins their exact scores, takes
 //                       every key above the bin of the k-th and ranks the
 //                       keys inside that bin (ties to the lower position).
@@ -157,6 +157,21 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
     const int s_end = min(s_begin + chunk_len, n_cand);
     const bool ranked = k > 0 && n_cand > k;
     if (ranked && s_end > s_begin) {
+        const float* srow = lrow + (size_t)b * score_ld;
+        // the first batch of L values is requested before the histogram is
+        // known (chunks start on 128-token boundaries; rows are padded to 4)
+        constexpr int U = 8;
+        float4 v[U];
+        auto load_batch = [&](int s0) {
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                const int s = s0 + u * 4 * kGatherThreads;
+                v[u] = s < s_end ? __ldcg(reinterpret_cast<const float4*>(srow + s))
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        };
+        int s0 = s_begin + 4 * (int)threadIdx.x;
+        load_batch(s0);
         if (warp == 0) {
             for (int i = lane; i < 256; i += 32) sh.hist[i] = (int)__ldcg(hist_g + b * 256 + i);
             __syncwarp();
@@ -167,11 +182,25 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
                 sh.n_cand = 0;
             }
         }
+        // f16-rounded query, 8 elements per thread
         const __nv_bfloat16* qb = q + (size_t)b * Hq * 128;
-        for (int e = threadIdx.x; e < 16 * 128; e += blockDim.x) {
+        for (int e = 8 * threadIdx.x; e < 16 * 128; e += 8 * kGatherThreads) {
             const int h = e >> 7;
-            sh.q[h][e & 127] =
-                h < Hq ? __half2float(__float2half_rn(__bfloat162float(qb[e]))) : 0.f;
+            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+            if (h < Hq) {
+                const uint4 w = *reinterpret_cast<const uint4*>(qb + e);
+                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    f[2 * i] = __half2float(__float2half_rn(bf16_lo(wd[i])));
+                    f[2 * i + 1] = __half2float(__float2half_rn(bf16_hi(wd[i])));
+                }
+                lo = make_float4(f[0], f[1], f[2], f[3]);
+                hi = make_float4(f[4], f[5], f[6], f[7]);
+            }
+            *reinterpret_cast<float4*>(&sh.q[h][e & 127]) = lo;
+            *reinterpret_cast<float4*>(&sh.q[h][(e & 127) + 4]) = hi;
         }
         __syncthreads();
         const int j = sh.bin;
@@ -182,18 +211,7 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
         const float E = j <= 0 ? 0.f : __uint_as_float(base + ((uint32_t)j << dec::kBinShift));
         const float eps = (float)Hq * 0x1p-23f;
         const float thr = (E - eps) * (8.f / 9.f) * (1.f - 0x1p-10f);
-        const float* srow = lrow + (size_t)b * score_ld;
-        // chunks start on 128-token boundaries; score rows are padded to 4;
-        // eight 16-byte loads in flight per thread
-        constexpr int U = 8;
-        for (int s0 = s_begin + 4 * (int)threadIdx.x; s0 < s_end; s0 += 4 * U * kGatherThreads) {
-            float4 v[U];
-#pragma unroll
-            for (int u = 0; u < U; u++) {
-                const int s = s0 + u * 4 * kGatherThreads;
-                v[u] = s < s_end ? __ldcg(reinterpret_cast<const float4*>(srow + s))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+        for (;;) {
 #pragma unroll
             for (int u = 0; u < U; u++) {
                 const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -206,37 +224,41 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
                     }
                 }
             }
+            s0 += 4 * U * kGatherThreads;
+            if (s0 - 4 * (int)threadIdx.x >= s_end) break;
+            load_batch(s0);
         }
         __syncthreads();
         const int nc = (int)sh.n_cand;
         if (nc > kCandCap) {
             if (threadIdx.x == 0) atomicOr(ovf + b, 1u);
         } else {
-            float l2[16];
-#pragma unroll
-            for (int h = 0; h < 16; h++) l2[h] = h < Hq ? __ldcg(lse2_ws + b * 16 + h) : INFINITY;
+            // a thread pair per candidate: lane & 1 takes dims 64 (lane & 1) .. + 63
+            const int half = lane & 1;
+            const int hh = (lane >> 1) & 15;  // the head this lane exponentiates
+            const float l2h = hh < Hq ? __ldcg(lse2_ws + b * 16 + hh) : INFINITY;
             const uint8_t* kb = kc + (size_t)b * Tmax * 128;
             const float* ksb = ksc + (size_t)b * Tmax;
-            for (int i0 = warp * 32; i0 < nc; i0 += kGatherThreads) {
-                const int i = i0 + lane;
+            for (int i0 = warp * 16; i0 < nc; i0 += kGatherThreads / 2) {
+                const int i = i0 + (lane >> 1);
                 const bool has = i < nc;
                 const int s = has ? sh.cand[i] : 0;
-                uint4 kw[8];
-                const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)s * 128);
+                uint4 kw[4];
+                const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)s * 128) + 4 * half;
 #pragma unroll
-                for (int c = 0; c < 8; c++) kw[c] = has ? __ldg(kr + c) : make_uint4(0u, 0u, 0u, 0u);
+                for (int c = 0; c < 4; c++) kw[c] = has ? __ldg(kr + c) : make_uint4(0u, 0u, 0u, 0u);
                 const float sk = has ? __ldg(ksb + s) : 0.f;
                 float d[16];
 #pragma unroll
                 for (int h = 0; h < 16; h++) d[h] = 0.f;
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
+                for (int c = 0; c < 4; c++) {
                     const uint32_t wd[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
 #pragma unroll
                     for (int m = 0; m < 4; m++) {
                         const float2 k01 = f16x2_to_float2(e4m3x2_lo_to_f16x2(wd[m]));
                         const float2 k23 = f16x2_to_float2(e4m3x2_lo_to_f16x2(wd[m] >> 16));
-                        const int dim = 16 * c + 4 * m;
+                        const int dim = 64 * half + 16 * c + 4 * m;
 #pragma unroll
                         for (int h = 0; h < 16; h++) {
                             const float4 qv = *reinterpret_cast<const float4*>(&sh.q[h][dim]);
@@ -247,16 +269,22 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
                         }
                     }
                 }
+                // whole dots on both lanes of the pair
+#pragma unroll
+                for (int h = 0; h < 16; h++) d[h] += __shfl_xor_sync(0xffffffffu, d[h], 1);
                 const float ks = sk * qk2;
                 float sc = 0.f;
 #pragma unroll
-                for (int h = 0; h < 16; h++) sc += ex2(fmaf(d[h], ks, -l2[h]));
-                // one boundary-buffer reservation per warp
-                const unsigned m = __ballot_sync(0xffffffffu, has);
+                for (int h = 0; h < 16; h++) {
+                    const float l2 = __shfl_sync(0xffffffffu, l2h, 2 * h);
+                    sc += ex2(fmaf(d[h], ks, -l2));
+                }
+                // one boundary-buffer reservation per warp (even lanes write)
+                const unsigned m = __ballot_sync(0xffffffffu, has && half == 0);
                 unsigned basep = 0;
                 if (lane == 0) basep = atomicAdd(bnd_cnt + b, (unsigned)__popc(m));
                 basep = __shfl_sync(0xffffffffu, basep, 0);
-                if (has) {
+                if (has && half == 0) {
                     const unsigned p = basep + (unsigned)__popc(m & ((1u << lane) - 1u));
                     if (p < (unsigned)dec::BCAP)
                         bnd[(size_t)b * dec::BCAP + p] = make_key(sc, (uint32_t)s);
