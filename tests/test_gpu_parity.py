@@ -81,6 +81,53 @@ def test_full_attn_select_matches_oracle(cuda_lib, shape):
     assert overlap > 0.999
 
 
+def _prefill_fail_flags(hs2, x, ws):
+    """Per query block, whether the speculative stream thresholds failed the
+    exact check (the workspace keeps them after the call: after the lse
+    scratch, one word per 128-row query block)."""
+    rows = x.B * x.L
+    off = (rows * x.q.shape[2] * 4 + 255) // 256 * 256
+    nqb = (x.L + 127) // 128
+    return ws[off: off + 4 * x.B * nqb].view(torch.int32).cpu().numpy()
+
+
+@pytest.mark.parametrize("decay", [0.0, 6.0])
+def test_full_attn_select_speculative_thresholds(cuda_lib, decay):
+    """Long rows (L = 8192, k = 256): the streams start from a speculative
+    threshold.  With exchangeable keys (decay 0) it holds; with key relevance
+    falling along the sequence (decay 6: early keys score higher) the first
+    sample overestimates it, the per-row check fails and the exact re-run of
+    those query blocks must give the same, exact selection."""
+    B, L, Hq, d, W, k = 1, 8192, 16, 128, 128, 256
+    x = inputs.make_prefill(B, L, Hq, d, W, k, n_topics=32, seg=256, seed=31, n_sparse=1)
+    if decay:
+        g = torch.Generator().manual_seed(32)
+        u = torch.randn(d, generator=g)
+        u /= u.norm()
+        ramp = decay * (1.0 - torch.arange(L, dtype=torch.float32) / L)
+        kf = x.k_.float() + ramp[None, :, None] * u
+        qf = x.q.float() + 3.0 * u
+        x = inputs.PrefillInputs(B, L, Hq, d, W, k, qf.bfloat16(), kf.bfloat16(), x.v, [],
+                                 None, None, None)
+    ws = torch.empty(cuda_lib.hs2_full_attn_select_workspace(
+        cuda_lib.prefill_shape(B, L, Hq, d, W, k)), dtype=torch.uint8, device="cuda")
+    o, lse, idx = cuda_lib.hs2_full_attn_select(cuda(x.q), cuda(x.k_), cuda(x.v), W, k,
+                                                workspace=ws)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    fails = _prefill_fail_flags(cuda_lib, x, ws)
+    if decay:
+        assert fails.sum() > 0, "the decaying keys should defeat the speculative thresholds"
+    idx = idx.cpu().numpy().reshape(B * L, -1)
+    t_all = np.tile(np.arange(L), B)
+    check_structure(idx, t_all, W, k)
+    rows = sample_rows(B, L, 192, seed=5)
+    ora = oracle.full_select(x.q, x.k_, x.v, W, k, rows=rows, probe=idx[rows])
+    o = o.float().cpu().numpy().reshape(B * L, Hq, d)
+    assert max_abs(o[rows], ora["o"]) <= TOL_BF16
+    check_selection(idx[rows], ora, rows % L, W, k)
+
+
 def test_full_attn_select_ties_take_lower_index(cuda_lib):
     """Keys drawn from 4 distinct rows: many exact score ties straddle the cut."""
     B, L, Hq, d, W, k = 1, 640, 16, 128, 16, 40
@@ -127,13 +174,19 @@ def test_sparse_attn_isolated_and_end_to_end(cuda_lib, kv):
 
 def test_sparse_equals_full_when_budget_covers(cuda_lib):
     """W+k >= L selects everything: the sparse layer with the full layer's own
-    queries must reproduce the full layer's output."""
+    queries must reproduce the full layer's output.  Both are bf16 roundings of
+    the same exact attention, each checked against the oracle; between them
+    the triangle bound 2 * TOL_BF16 applies (two roundings of one value can
+    differ by an ulp, 2^-6 for |o| in [2, 4))."""
     B, L, Hq, d, W, k = 1, 200, 16, 128, 8, 200
     x = inputs.make_prefill(B, L, Hq, d, W, k, seed=5)
     o, _, idx = cuda_lib.hs2_full_attn_select(cuda(x.q), cuda(x.k_), cuda(x.v), W, k)
     o2 = cuda_lib.hs2_sparse_attn(cuda(x.q), cuda(x.k_), cuda(x.v), idx, W=W, k_top=k)
     torch.cuda.synchronize()
-    assert (o.float() - o2.float()).abs().max().item() <= TOL_BF16
+    ora = oracle.full_select(x.q, x.k_, x.v, W, k)
+    assert max_abs(o.float().cpu().numpy().reshape(B * L, Hq, d), ora["o"]) <= TOL_BF16
+    assert max_abs(o2.float().cpu().numpy().reshape(B * L, Hq, d), ora["o"]) <= TOL_BF16
+    assert (o.float() - o2.float()).abs().max().item() <= 2 * TOL_BF16
 
 
 def test_sparse_attn_flags_out_of_range_indices(cuda_lib):

@@ -184,13 +184,16 @@ bool map_kv(CUtensorMap* m, const void* x, int B, int L, int D, int rows) {
 int pf_cap(int k) { return (int)round_up((size_t)2 * k + 128, 32); }
 
 struct PrefillWs {
-    size_t lse_off, buf_off, total;
+    size_t lse_off, fail_off, fail_bytes, buf_off, total;
 };
 PrefillWs prefill_ws(const hs2_prefill_shape* s) {
     PrefillWs w;
     const size_t rows = (size_t)s->B * s->L;
     w.lse_off = 0;
-    w.buf_off = round_up(rows * s->Hq * sizeof(float), 256);
+    // per query block: the speculative selection's check failed (zeroed per call)
+    w.fail_off = round_up(rows * s->Hq * sizeof(float), 256);
+    w.fail_bytes = (size_t)s->B * ((s->L + tcfa::BM - 1) / tcfa::BM) * sizeof(unsigned);
+    w.buf_off = round_up(w.fail_off + w.fail_bytes, 256);
     w.total = w.buf_off + (s->k > 0 ? rows * 2 * pf_cap(s->k) * sizeof(uint64_t) : 0);
     return w;
 }
@@ -224,9 +227,16 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
         auto kern = tcfa::prefill_select_tc_kernel<D>;
         if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
         dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->B);
+        unsigned* fail = reinterpret_cast<unsigned*>(ws + w.fail_off);
+        uint64_t* buf = reinterpret_cast<uint64_t*>(ws + w.buf_off);
+        if (cudaMemsetAsync(fail, 0, w.fail_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
+        // speculative thresholds, then the exact selection for the query blocks
+        // whose rows failed the check (a gated launch: the others return at once)
         kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
-                                      pf_cap(s->k), scale2,
-                                      reinterpret_cast<uint64_t*>(ws + w.buf_off), idx, flags);
+                                      pf_cap(s->k), scale2, buf, idx, 1, nullptr, fail, flags);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
+                                      pf_cap(s->k), scale2, buf, idx, 0, fail, nullptr, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     return HS2_OK;

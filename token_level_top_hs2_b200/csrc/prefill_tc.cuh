@@ -210,7 +210,7 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const uint32_t s_col = lane_base + (hh ? F::COL_S1 : F::COL_S0);
         const uint32_t o_col = lane_base + (hh ? F::COL_O1 : F::COL_O0);
-        float m = -INFINITY, l = 0.f;
+        float m = -INFINITY, l = 0.f, lq = 0.f;
         bool ok = true;
         for (int j = 0; j < n_kt; j++) {
             if (!mbar_wait(&bars.s_full[hh], j & 1, abort_, flags)) {
@@ -227,7 +227,8 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
 #pragma unroll
                 for (int i = 0; i < 32; i++) x[c * 32 + i] = __uint_as_float(r[i]) * scale2;
             }
-            if (j == n_kt - 1) {  // diagonal tile: keys j*128 + i, row t = qb*128 + row
+            const bool diag = j == n_kt - 1;
+            if (diag) {  // diagonal tile: keys j*128 + i, row t = qb*128 + row
 #pragma unroll
                 for (int i = 0; i < BN; i++)
                     if (i > row) x[i] = -INFINITY;
@@ -239,6 +240,7 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (j > 0) {
                     const float alpha = ex2(m - mx);
                     l *= alpha;
+                    lq *= alpha;
                     // O holds the sum up to tile j-1: wait for that PV, rescale in TMEM
                     if (!mbar_wait(&bars.o_done[hh], (j - 1) & 1, abort_, flags)) {
                         ok = false;
@@ -258,7 +260,7 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
                 m = mx;
             }
-            float rs = 0.f;
+            float rs = 0.f, rq = 0.f;
 #pragma unroll
             for (int c = 0; c < BN / 32; c++) {
                 uint32_t w[16];
@@ -268,9 +270,16 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     rs += p0 + p1;
                     w[i] = pack_bf16(p0, p1);
                 }
+                // the diagonal tile (early rows: all their keys) also sums the
+                // bf16 weights the PV product uses, to normalise O by them
+                if (diag) {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) rq += bf16_lo(w[i]) + bf16_hi(w[i]);
+                }
                 tmem_st16(s_col + c * 16, w);
             }
             l += rs;
+            lq += diag ? rq : rs;
             tmem_st_wait();
             fence_before_sync();
             __syncwarp();
@@ -280,7 +289,10 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         if (ok && mbar_wait(&bars.o_done[hh], (n_kt - 1) & 1, abort_, flags)) {
             fence_after_sync();
             const int h = h0 + hh;
-            const float inv = 1.f / l;
+            // O is normalised by lq, in which the diagonal tile counts the bf16
+            // weights the PV product used (for rows below 128 those are all of
+            // their weights, which then sum to exactly one); lse uses the exact sum
+            const float inv = 1.f / lq;
             const bool store = t < L;
             __nv_bfloat16* orow = o + (((size_t)b * L + (store ? t : 0)) * Hq + h) * D;
 #pragma unroll
@@ -377,6 +389,32 @@ HS2_DEV int rel_bin(uint32_t bits, uint32_t base) {
 // batch are in flight together (the lists live in DRAM-backed workspace).
 constexpr int kBatch = 8;
 
+// Keep, in place and in order, the keys of a stream buffer whose score bits
+// are >= tb (one warp); returns their count.  A batch is fully read before any
+// of its writes, and writes never pass the end of the batch.
+HS2_DEV int warp_keep_bits(uint64_t* buf, int cnt, uint32_t tb) {
+    const int lane = lane_id();
+    int wp = 0;
+    for (int i0 = 0; i0 < cnt; i0 += 32 * kBatch) {
+        uint64_t v[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int i = i0 + u * 32 + lane;
+            v[u] = i < cnt ? __ldcg(buf + i) : 0;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; u++) {
+            const int i = i0 + u * 32 + lane;
+            const bool kp = i < cnt && (uint32_t)(v[u] >> 32) >= tb;
+            const unsigned bal = __ballot_sync(0xffffffffu, kp);
+            if (kp) __stcg(buf + wp + __popc(bal & ((1u << lane) - 1)), v[u]);
+            wp += __popc(bal);
+        }
+    }
+    __syncwarp();
+    return wp;
+}
+
 HS2_DEV int warp_prune(uint64_t* buf, int cnt, int k, int room, uint32_t base, int* hist,
                        uint32_t* tb_out) {
     const int lane = lane_id();
@@ -404,28 +442,8 @@ HS2_DEV int warp_prune(uint64_t* buf, int cnt, int k, int room, uint32_t base, i
     const int keep = above + in_bin;
     if (j < 0 || keep > room) return -1;
     const uint32_t tb = base + ((uint32_t)j << kBinShift);
-    // in-place compaction: a batch is fully read before any of its writes,
-    // and writes never pass the end of the batch
-    int wp = 0;
-    for (int i0 = 0; i0 < cnt; i0 += 32 * kBatch) {
-        uint64_t v[kBatch];
-#pragma unroll
-        for (int u = 0; u < kBatch; u++) {
-            const int i = i0 + u * 32 + lane;
-            v[u] = i < cnt ? __ldcg(buf + i) : 0;
-        }
-#pragma unroll
-        for (int u = 0; u < kBatch; u++) {
-            const int i = i0 + u * 32 + lane;
-            const bool kp = i < cnt && (uint32_t)(v[u] >> 32) >= tb;
-            const unsigned bal = __ballot_sync(0xffffffffu, kp);
-            if (kp) __stcg(buf + wp + __popc(bal & ((1u << lane) - 1)), v[u]);
-            wp += __popc(bal);
-        }
-    }
-    __syncwarp();
     *tb_out = tb;
-    return wp;
+    return warp_keep_bits(buf, cnt, tb);
 }
 
 // Cut a stream buffer of `cnt` unique keys to its k best in place (one warp,
@@ -454,7 +472,9 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                          const __grid_constant__ CUtensorMap map_k,
                          const float* __restrict__ lse, int L, int Hq, int W, int kk, int S,
                          int cap, float scale2, uint64_t* __restrict__ wsbuf,
-                         int32_t* __restrict__ idx, unsigned* __restrict__ flags) {
+                         int32_t* __restrict__ idx, int speculate,
+                         const unsigned* __restrict__ gate, unsigned* __restrict__ fail_qb,
+                         unsigned* __restrict__ flags) {
     using F = Sel<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -464,6 +484,8 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     const int nqb = (L + BM - 1) / BM;
     const int qb = nqb - 1 - (int)blockIdx.x;
     const int b = blockIdx.y;
+    // the exact re-run only redoes the query blocks whose check failed
+    if (gate != nullptr && __ldg(gate + (size_t)b * nqb + qb) == 0u) return;
     const int last_key = (kk > 0) ? min(qb * BM + BM, L) - 1 - W : -1;  // candidates 0..last_key
     const int n_kb = last_key >= 0 ? last_key / SBN + 1 : 0;
     const int n_it = n_kb * Hq;
@@ -580,6 +602,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 score warps
         int cnt = 0;
         uint32_t thr_bits = 0;  // appended keys have score bits >= thr_bits
+        bool pruned = false;    // the stream has had its first prune
         // histogram origin of a stream's first prune: 1/64 of the row's mean
         // score Hq/(t+1); later prunes start from the stream's threshold
         const uint32_t base_bits = __float_as_uint((float)Hq / (64.f * (float)(t + 1)));
@@ -598,7 +621,20 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     const int scnt = __shfl_sync(0xffffffffu, cnt, src);
                     const uint32_t sbase = __shfl_sync(0xffffffffu, max(thr_bits, base_bits), src);
                     uint32_t ntb = 0;
-                    int ncnt = warp_prune(sbuf, scnt, kk, cap - 128, sbase, hist, &ntb);
+                    int ncnt = -1;
+                    if (speculate && !__shfl_sync(0xffffffffu, pruned, src)) {
+                        // first prune: every candidate so far is buffered (threshold
+                        // 0), a sample of scnt of the row's n_row candidates; keep
+                        // about twice its expected share of the row's top k
+                        const int n_row = __shfl_sync(0xffffffffu, maxkey + 1, src);
+                        const long long r = 2LL * kk * scnt / max(n_row, 1) + 64;
+                        // (the histogram prune keeps every key whose score bits
+                        // reach the bin of the r-th best; if that frees no room
+                        // the buffer is left as it was and pruned to k below)
+                        if (r < kk)
+                            ncnt = warp_prune(sbuf, scnt, (int)r, cap - 128, sbase, hist, &ntb);
+                    }
+                    if (ncnt < 0) ncnt = warp_prune(sbuf, scnt, kk, cap - 128, sbase, hist, &ntb);
                     if (ncnt < 0) {  // no histogram boundary frees room: exact cut to k
                         const uint64_t nthr = warp_cut(sbuf, scnt, kk, hist);
                         ntb = (uint32_t)(nthr >> 32);
@@ -607,6 +643,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     if (lane == src) {
                         thr_bits = ntb;
                         cnt = ncnt;
+                        pruned = true;
                     }
                 }
             }
@@ -681,6 +718,19 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             int32_t* out = idx + ((size_t)b * L + t) * S;
             for (int i = lane; i < wl; i += 32) out[i] = w0 + i;
             int wp = wl;
+            const uint32_t base = max(tbs[row], tbs[128 + row]);
+            if (speculate) {
+                // every key whose score bits reach `base` is in the union; the
+                // row is exact iff at least min(k, candidates) of them are
+                int ge = 0;
+                for (int i = lane; i < n; i += 32) ge += (uint32_t)(get(i) >> 32) >= base;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ge += __shfl_xor_sync(0xffffffffu, ge, o);
+                if (ge < min(kk, max(0, t - W + 1))) {
+                    if (lane == 0) atomicOr(fail_qb + (size_t)b * nqb + qb, 1u);
+                    continue;  // the exact re-run writes this row
+                }
+            }
             if (n <= kk) {
                 for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
                     uint64_t v[kBatch];
@@ -697,7 +747,6 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
                 wp += n;
             } else {
-                const uint32_t base = max(tbs[row], tbs[128 + row]);
 #pragma unroll
                 for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
                 __syncwarp();
