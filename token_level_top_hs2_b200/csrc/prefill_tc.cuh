@@ -338,9 +338,15 @@ namespace tcfa {
 // 128..255) add 2^(S*scale*log2e - lse2_h) into 128 registers; after the last
 // head they hold score(t, s) for their 128 keys and feed the candidates
 // (s <= t-W) into the (row, half) stream: keys >= the stream's threshold are
-// appended to its workspace buffer; a buffer that would overflow is cut to its
-// k best by a warp radix select (one lane's buffer at a time), raising the
-// threshold.  At the end the two streams of a row are merged to exactly k.
+// appended to its workspace buffer.  A buffer that would overflow is pruned
+// (one lane's buffer at a time) by a score-bit histogram.  A speculative prune
+// keeps only the keys reaching about 1.5 times the stream's expected share of
+// the row's top k, so the threshold approaches the row's final k-th score
+// early and few candidates are appended; if no bin boundary frees room, the
+// buffer is cut to about its k best (or exactly, by a radix select).  At the
+// end the two streams of a row are merged to exactly k, after an exact check
+// (at least min(k, candidates) keys reach the higher stream threshold); rows
+// that fail it flag their query block for a gated exact re-run.
 // The L x L score matrix never leaves the chip.
 constexpr int SBN = 256;   // keys per block
 constexpr int QSTAGE = 2;
@@ -602,7 +608,6 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 score warps
         int cnt = 0;
         uint32_t thr_bits = 0;  // appended keys have score bits >= thr_bits
-        bool pruned = false;    // the stream has had its first prune
         // histogram origin of a stream's first prune: 1/64 of the row's mean
         // score Hq/(t+1); later prunes start from the stream's threshold
         const uint32_t base_bits = __float_as_uint((float)Hq / (64.f * (float)(t + 1)));
@@ -622,12 +627,14 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     const uint32_t sbase = __shfl_sync(0xffffffffu, max(thr_bits, base_bits), src);
                     uint32_t ntb = 0;
                     int ncnt = -1;
-                    if (speculate && !__shfl_sync(0xffffffffu, pruned, src)) {
-                        // first prune: every candidate so far is buffered (threshold
-                        // 0), a sample of scnt of the row's n_row candidates; keep
-                        // about twice its expected share of the row's top k
+                    if (speculate) {
+                        // the stream has seen kb*128 of the row's n_row candidates
+                        // and buffers every one of them at or above its threshold;
+                        // keep 1.5 times their expected share of the row's top k,
+                        // plus 32 (on the planted-topic workloads no row failed
+                        // the exact check at this margin; at 1.25x + 16 a few did)
                         const int n_row = __shfl_sync(0xffffffffu, maxkey + 1, src);
-                        const long long r = 2LL * kk * scnt / max(n_row, 1) + 64;
+                        const long long r = 3LL * kk * (kb * 128) / (2LL * max(n_row, 1)) + 32;
                         // (the histogram prune keeps every key whose score bits
                         // reach the bin of the r-th best; if that frees no room
                         // the buffer is left as it was and pruned to k below)
@@ -643,7 +650,6 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     if (lane == src) {
                         thr_bits = ntb;
                         cnt = ncnt;
-                        pruned = true;
                     }
                 }
             }
