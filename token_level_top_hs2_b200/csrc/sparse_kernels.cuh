@@ -131,9 +131,12 @@ decode_sparse_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restr
     merge_partials_block<D>(wpart + 16 * D, wpart + 16 * D + 16, wpart, WARPS, PART, PART, Hq,
                             cpart + 16 * D, cpart + 16 * D + 16, cpart);
     cluster.sync();
-    if (rank == 0) {
-        // gather the CLUSTER merged partials through distributed shared memory
-        for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
+    {
+        // merge the CLUSTER partials through distributed shared memory; each
+        // CTA of the cluster produces its own slice of the Hq x D outputs
+        const int per = (Hq * D + CLUSTER - 1) / CLUSTER;
+        const int e1 = min(Hq * D, (rank + 1) * per);
+        for (int e = rank * per + (int)threadIdx.x; e < e1; e += blockDim.x) {
             const int row = e / D;
             float mx = -INFINITY;
             for (int r = 0; r < CLUSTER; r++) {
