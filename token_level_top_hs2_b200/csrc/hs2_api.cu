@@ -517,7 +517,7 @@ hs2_status run_decode_sparse(const hs2_decode_shape* s, const void* q, const voi
                              const void* vc, const float* ks, const float* vs,
                              const int32_t* lengths, const int32_t* idx, void* o,
                              cudaStream_t st, unsigned* flags) {
-    constexpr int WARPS = 4, CLUSTER = 8;
+    constexpr int WARPS = 6, CLUSTER = 8;
     const size_t smem = (size_t)(WARPS + 1) * (16 * D + 32) * sizeof(float);
     auto kern = decode_sparse_kernel<D, FP8, WARPS, CLUSTER>;
     if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
