@@ -34,6 +34,14 @@ enum : unsigned {
 
 HS2_DEV uint32_t lane_id() { return threadIdx.x & 31; }
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialisation may start while the kernel before it in the stream still
+// runs: griddep_wait() returns once that kernel has completed and its memory
+// is visible; griddep_launch() lets the next kernel of the stream start
+// launching.  Both are no-ops in a kernel launched the plain way.
+HS2_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+HS2_DEV void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 HS2_DEV float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -118,6 +118,9 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     float* skb = reinterpret_cast<float*>(smem + LY::OFF_SC);  // [kDK][128]
     float* svb = skb + kDK * TOK;                              // [kDK][128]
     float* red = reinterpret_cast<float*>(smem + LY::OFF_RED); // [4][16]
+    // the selection kernels that follow may launch now; they wait for this
+    // grid to complete before reading what it writes
+    griddep_launch();
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kNR; i++) {
@@ -484,7 +487,11 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // ---- the last chunk of the sequence merges every chunk's partial
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) bars.last = (atomicAdd(counter + b, 1u) == (unsigned)(n_chunks - 1));
+    if (threadIdx.x == 0) {
+        // the per-call counters are zeroed by the kernel launched before this one
+        griddep_wait();
+        bars.last = (atomicAdd(counter + b, 1u) == (unsigned)(n_chunks - 1));
+    }
     __syncthreads();
     if (!bars.last) return;
     __threadfence();

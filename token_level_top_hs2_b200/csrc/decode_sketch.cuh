@@ -52,11 +52,14 @@ sketch_score_kernel(const uint8_t* __restrict__ sketch, const float* __restrict_
                     int score_ld, unsigned* __restrict__ hist_g) {
     // one counter column per lane: the lanes of a warp never collide
     __shared__ unsigned hist[256 * 32];
+    griddep_launch();
     const int b = blockIdx.y;
     const int T = __ldg(lengths + b);
     const int n_cand = (T >= 1 && T <= Tmax) ? max(0, T - W) : 0;
-    if (k <= 0 || n_cand <= k) return;
     for (int i = threadIdx.x; i < 256 * 32; i += blockDim.x) hist[i] = 0;
+    // the sketch, the tile references and lse2 come from the kernel before
+    griddep_wait();
+    if (k <= 0 || n_cand <= k) return;
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = lane_id();
     constexpr int NW = kScoreThreads / 32;
@@ -156,7 +159,33 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
     const int s_begin = chunk * chunk_len;
     const int s_end = min(s_begin + chunk_len, n_cand);
     const bool ranked = k > 0 && n_cand > k;
-    if (ranked && s_end > s_begin) {
+    const bool work = ranked && s_end > s_begin;
+    griddep_launch();
+    if (work) {
+        // f16-rounded query, 8 elements per thread
+        const __nv_bfloat16* qb = q + (size_t)b * Hq * 128;
+        for (int e = 8 * threadIdx.x; e < 16 * 128; e += 8 * kGatherThreads) {
+            const int h = e >> 7;
+            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
+            if (h < Hq) {
+                const uint4 w = *reinterpret_cast<const uint4*>(qb + e);
+                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+                float f[8];
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    f[2 * i] = __half2float(__float2half_rn(bf16_lo(wd[i])));
+                    f[2 * i + 1] = __half2float(__float2half_rn(bf16_hi(wd[i])));
+                }
+                lo = make_float4(f[0], f[1], f[2], f[3]);
+                hi = make_float4(f[4], f[5], f[6], f[7]);
+            }
+            *reinterpret_cast<float4*>(&sh.q[h][e & 127]) = lo;
+            *reinterpret_cast<float4*>(&sh.q[h][(e & 127) + 4]) = hi;
+        }
+    }
+    // L, its histogram and lse2 come from the kernels before
+    griddep_wait();
+    if (work) {
         const float* srow = lrow + (size_t)b * score_ld;
         // the first batch of L values is requested before the histogram is
         // known (chunks start on 128-token boundaries; rows are padded to 4)
@@ -181,26 +210,6 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
                 sh.bin = j;
                 sh.n_cand = 0;
             }
-        }
-        // f16-rounded query, 8 elements per thread
-        const __nv_bfloat16* qb = q + (size_t)b * Hq * 128;
-        for (int e = 8 * threadIdx.x; e < 16 * 128; e += 8 * kGatherThreads) {
-            const int h = e >> 7;
-            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
-            if (h < Hq) {
-                const uint4 w = *reinterpret_cast<const uint4*>(qb + e);
-                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    f[2 * i] = __half2float(__float2half_rn(bf16_lo(wd[i])));
-                    f[2 * i + 1] = __half2float(__float2half_rn(bf16_hi(wd[i])));
-                }
-                lo = make_float4(f[0], f[1], f[2], f[3]);
-                hi = make_float4(f[4], f[5], f[6], f[7]);
-            }
-            *reinterpret_cast<float4*>(&sh.q[h][e & 127]) = lo;
-            *reinterpret_cast<float4*>(&sh.q[h][(e & 127) + 4]) = hi;
         }
         __syncthreads();
         const int j = sh.bin;

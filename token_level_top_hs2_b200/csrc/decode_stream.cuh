@@ -380,7 +380,9 @@ gather_kernel(const float* __restrict__ scores, int score_ld, const unsigned* __
     extern __shared__ uint64_t sk[];  // BCAP keys (last CTA)
     __shared__ GatherShared sh;
     const int b = blockIdx.y, chunk = blockIdx.x;
-    if (gate != nullptr && __ldg(gate + b) == 0u) return;
+    // the scores, their histogram and the gate come from the kernels before
+    griddep_wait();
+    if (gate != nullptr && __ldcg(gate + b) == 0u) return;
     const int T = __ldg(lengths + b);
     const bool ok = T >= 1 && T <= Tmax;
     const int n_cand = ok ? max(0, T - W) : 0;

@@ -177,8 +177,11 @@ pass2_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     __shared__ Bars bars;
     __shared__ unsigned hist[256];
     const int b = blockIdx.y, chunk = blockIdx.x;
-    // run only for the sequences the sketch selection handed over, if gated
-    if (gate != nullptr && __ldg(gate + b) == 0u) return;
+    // run only for the sequences the sketch selection handed over, if gated;
+    // the gate (and lse2) come from the kernels before
+    griddep_launch();
+    griddep_wait();
+    if (gate != nullptr && __ldcg(gate + b) == 0u) return;
     const int warp = threadIdx.x >> 5, lane = lane_id();
     const int T = __ldg(lengths + b);
     const int n_cand = (T >= 1 && T <= Tmax) ? max(0, T - W) : 0;

@@ -106,6 +106,33 @@ bool set_smem(K kernel, size_t bytes) {
     return true;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel of the stream drains (its prologue overlaps that
+// kernel's tail); it calls griddep_wait() before reading that kernel's
+// results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Zeroes n16 16-byte words; lets the next kernel of the stream launch at once.
+__global__ void zero16_kernel(uint4* __restrict__ p, int n16) {
+    griddep_launch();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n16; i += gridDim.x * blockDim.x)
+        p[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
 // ------------------------------------------------------------ tensor maps
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no direct
 // libcuda link).  bf16 tensors, 128-byte swizzle, 64-element inner box.
@@ -382,9 +409,13 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
         mks = mk;  // unused placeholders
         mvs = mk;
     }
-    if (cudaMemsetAsync(zero, 0, w.zero_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
     const auto* qp = static_cast<const __nv_bfloat16*>(q);
     if constexpr (FP8 && D == 128) {
+        // a chain of launches with programmatic serialisation: each kernel's
+        // launch and prologue overlap the tail of the one before
+        const int n16 = (int)(w.zero_bytes / 16);  // zero_bytes = B * 2080
+        zero16_kernel<<<(n16 + 255) / 256, 256, 0, st>>>(reinterpret_cast<uint4*>(zero), n16);
+        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
         // tensor-memory path: tokens as the MMA M dimension, exact f16 K/V
         const float qk2 = s->scale * kLog2e;
         using LY = dtc::P1Layout;
@@ -393,33 +424,37 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
         uint8_t* skt = sketch ? ws + w.sketch_off : nullptr;
         float* rsnap = reinterpret_cast<float*>(ws + w.rsnap_off);
         if (!set_smem(dtc::pass1_tc_kernel, LY::SMEM)) return HS2_ERR_CUDA;
-        dtc::pass1_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kP1Threads, LY::SMEM, st>>>(
-            mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len, w.n_chunks, qk2, part,
-            cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o), skt, rsnap, w.sk_tiles, flags);
-        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        if (launch_pdl(dtc::pass1_tc_kernel, dim3(w.n_chunks, s->B), dim3(dtc::kP1Threads),
+                       LY::SMEM, st, mk, mv, mks, mvs, qp, lengths, s->Tmax, s->Hq, w.chunk_len,
+                       w.n_chunks, qk2, part, cnt1, lse2, lse, static_cast<__nv_bfloat16*>(o),
+                       skt, rsnap, w.sk_tiles, flags) != cudaSuccess)
+            return HS2_ERR_CUDA;
         if (sketch) {
             // three resident CTAs per SM over the whole batch, one wave
             const int g_sc = 3 * 148 / s->B > 0 ? 3 * 148 / s->B : 1;
-            dsk::sketch_score_kernel<<<dim3(g_sc, s->B), dsk::kScoreThreads, 0, st>>>(
-                skt, rsnap, w.sk_tiles, lengths, s->Tmax, s->Hq, s->W, s->k, lse2, scores,
-                w.score_ld, sk_hist);
-            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+            if (launch_pdl(dsk::sketch_score_kernel, dim3(g_sc, s->B), dim3(dsk::kScoreThreads),
+                           0, st, skt, rsnap, w.sk_tiles, lengths, s->Tmax, s->Hq, s->W, s->k,
+                           lse2, scores, w.score_ld, sk_hist) != cudaSuccess)
+                return HS2_ERR_CUDA;
             const size_t smem = (size_t)dec::BCAP * sizeof(uint64_t);
             if (!set_smem(dsk::sketch_gather_kernel, smem)) return HS2_ERR_CUDA;
-            dsk::sketch_gather_kernel<<<dim3(w.n_chunks, s->B), dsk::kGatherThreads, smem, st>>>(
-                scores, w.score_ld, sk_hist, static_cast<const uint8_t*>(kc), ks, qp, lse2, qk2,
-                lengths, s->Tmax, s->Hq, s->W, s->k, w.chunk_len, w.n_chunks, sk_bnd, bnd, sk_ovf,
-                sk_cnt, idx);
-            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+            if (launch_pdl(dsk::sketch_gather_kernel, dim3(w.n_chunks, s->B),
+                           dim3(dsk::kGatherThreads), smem, st, scores, w.score_ld, sk_hist,
+                           static_cast<const uint8_t*>(kc), ks, qp, lse2, qk2, lengths, s->Tmax,
+                           s->Hq, s->W, s->k, w.chunk_len, w.n_chunks, sk_bnd, bnd, sk_ovf,
+                           sk_cnt, idx) != cudaSuccess)
+                return HS2_ERR_CUDA;
             // sequences whose candidates overflowed: exact scores, then the exact gather
             if (!set_smem(dtc::pass2_tc_kernel, LY2::SMEM)) return HS2_ERR_CUDA;
-            dtc::pass2_tc_kernel<<<dim3(w.n_chunks, s->B), dtc::kThreads, LY2::SMEM, st>>>(
-                mk, mks, qp, lengths, s->Tmax, s->Hq, s->W, w.chunk_len, qk2, lse2, scores,
-                w.score_ld, hist, sk_ovf, flags);
-            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+            if (launch_pdl(dtc::pass2_tc_kernel, dim3(w.n_chunks, s->B), dim3(dtc::kThreads),
+                           LY2::SMEM, st, mk, mks, qp, lengths, s->Tmax, s->Hq, s->W,
+                           w.chunk_len, qk2, lse2, scores, w.score_ld, hist,
+                           static_cast<const unsigned*>(sk_ovf), flags) != cudaSuccess)
+                return HS2_ERR_CUDA;
         }
         gate = sketch ? sk_ovf : nullptr;
     } else {
+        if (cudaMemsetAsync(zero, 0, w.zero_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
         auto kern = dec::pass1_kernel<D, FP8>;
         if (!set_smem(kern, SG::SMEM1)) return HS2_ERR_CUDA;
         kern<<<dim3(w.n_chunks, s->B), dec::kThreads, SG::SMEM1, st>>>(
@@ -438,10 +473,12 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     {
         const size_t smem = (size_t)dec::BCAP * sizeof(uint64_t);
         if (!set_smem(dec::gather_kernel, smem)) return HS2_ERR_CUDA;
-        dec::gather_kernel<<<dim3(w.n_chunks, s->B), 256, smem, st>>>(
-            scores, w.score_ld, hist, lengths, s->Tmax, s->Hq, s->W, s->k, w.chunk_len, w.n_chunks,
-            out_cnt, bnd_cnt, bnd, cnt3, idx, gate);
-        if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+        // waits for the kernel before at its top, whichever path launched it
+        if (launch_pdl(dec::gather_kernel, dim3(w.n_chunks, s->B), dim3(256), smem, st, scores,
+                       w.score_ld, static_cast<const unsigned*>(hist), lengths, s->Tmax, s->Hq,
+                       s->W, s->k, w.chunk_len, w.n_chunks, out_cnt, bnd_cnt, bnd, cnt3, idx,
+                       gate) != cudaSuccess)
+            return HS2_ERR_CUDA;
     }
     return HS2_OK;
 }
