@@ -242,20 +242,33 @@ def run_ours(args, world, rank, local):
         for j in range(ndsp):
             dsp(j)
 
+    # cross-layer overlap (diagnostic): the inherited selection against the one
+    # the first sparse layer's own queries give, made once outside the timing
+    idx_own = torch.empty_like(idx)
+    inter = torch.empty(B, L, dtype=torch.int32, device=dev)
+    ratio = torch.empty(B, L, dtype=torch.float32, device=dev)
+    hs2.hs2_full_attn_select(qs[0], k, v, W, K, o=os_, lse=lse, idx=idx_own, workspace=ws)
+
+    def overlap():
+        hs2.hs2_selection_overlap(idx, idx_own, W, K, inter=inter, ratio=ratio)
+
     pieces = [("full_select", full)] + [(f"sparse{j}", (lambda j=j: sparse(j)))
                                          for j in range(nsp)]
     pieces += [("decode_select", dsel)] + [(f"decode_sparse{j}", (lambda j=j: dsp(j)))
                                           for j in range(ndsp)]
-    # kernels per call: full select 2 (pass 1, pass 2 + selection); sparse 1;
-    # decode select 5 (pass 1, sketch score, sketch gather, and the exact
-    # pass 2 and gather, launched gated: they return at once unless a sequence
-    # overflowed the sketch candidates); decode sparse 1
-    dsel_launches = 5
-    launches_per_step = 2 + nsp + dsel_launches + ndsp
+    # kernels per call: full select 3 (pass 1, pass 2 + selection, and pass 2
+    # again gated: it returns at once unless a query block failed the check of
+    # its speculative thresholds); sparse 1; decode select 6 (workspace zeroing,
+    # pass 1, sketch score, sketch gather, and the exact pass 2 and gather,
+    # gated: they return at once unless a sequence overflowed the sketch
+    # candidates); decode sparse 1; overlap 1
+    full_launches, dsel_launches = 3, 6
+    launches_per_step = full_launches + nsp + dsel_launches + ndsp + 1
 
     for _ in range(args.warmup):
         for _, fn in pieces:
             fn()
+        overlap()
     # decode step as one CUDA graph (launch-bound inner loop)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -266,6 +279,7 @@ def run_ours(args, world, rank, local):
 
     times = {name: [] for name, _ in pieces}
     times["decode_step_graph"] = []
+    times["overlap"] = []
     barrier(world)
     with Clocks(local, not args.no_clocks) as clk:
         barrier(world)
@@ -285,6 +299,12 @@ def run_ours(args, world, rank, local):
             g.replay()
             e1.record(stream)
             evs.append(("decode_step_graph", e0, e1))
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            overlap()
+            e1.record(stream)
+            evs.append(("overlap", e0, e1))
             torch.cuda.synchronize()
             for name, a, b in evs:
                 times[name].append(a.elapsed_time(b))
@@ -299,6 +319,7 @@ def run_ours(args, world, rank, local):
     t_dsel = ms["decode_select"] / 1e3
     t_dsp = sum(ms[f"decode_sparse{j}"] for j in range(ndsp)) / ndsp / 1e3
     t_dstep = ms["decode_step_graph"] / 1e3
+    t_ovl = ms["overlap"] / 1e3
     ms_per_step = sum(ms[n] for n, _ in pieces)
 
     value = world * B * L / t_full
@@ -306,6 +327,7 @@ def run_ours(args, world, rank, local):
     sbytes = sparse_bytes(L, S, d) * B
     dbytes = decode_bytes(Bd, T, dd)
     dsp_bytes = float(Bd) * (xd.W + xd.k) * (2 * dd + 8)
+    ovl_bytes = float(B) * L * (2 * S * 4 + 8)
 
     def roof(kernel, bound, work, t, peak, unit, peak_src):
         ach = work / t / (1e12 if unit == "TFLOP/s" else 1e9)
@@ -320,12 +342,15 @@ def run_ours(args, world, rank, local):
         roof("sparse_attn", "hbm", sbytes, t_sparse, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
         roof("decode_select", "hbm", dbytes, t_dsel, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
         roof("decode_sparse", "hbm", dsp_bytes, t_dsp, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
+        roof("selection_overlap", "hbm", ovl_bytes, t_ovl, P["hbm"], "GB/s",
+             f"hbm_gbs ({P['src']})"),
     ]
     kernels[0]["frac_of_burst_peak"] = round(kernels[0]["achieved"] / P["bf16"], 4)
     kernels[0]["work"] = "3*d*Hq*L*(L+1) flops (pass 1 QK^T+PV, pass 2 QK^T)"
     kernels[1]["work"] = "sum_t min(t+1,S)*2*d*2 logical gathered bytes"
     kernels[2]["work"] = "B*T*(2d+8) bytes (e4m3 K,V rows + 2 fp32 scales)"
     kernels[3]["work"] = "B*S*(2d+8) bytes"
+    kernels[4]["work"] = "B*L*(2*S*4 + 8) bytes (two idx rows in, count and ratio out)"
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -343,14 +368,17 @@ def run_ours(args, world, rank, local):
             "decode_us_per_step_unfused_calls": round((t_dsel + ndsp * t_dsp) * 1e6, 1),
             "decode_select_us": round(t_dsel * 1e6, 1),
             "decode_sparse_us": round(t_dsp * 1e6, 1),
+            "selection_overlap_us": round(t_ovl * 1e6, 1),
+            "selection_overlap_mean": round(float(ratio.double().mean()), 4),
             "ms": {n: round(x, 4) for n, x in ms.items()},
         },
         "roofline": kernels[0],
         "kernels": kernels,
         "gpu_launches": launches_per_step * args.steps + (dsel_launches + ndsp) * args.steps,
-        "gpu_launches_note": f"per step: 2 full-select + {nsp} sparse + {dsel_launches} "
-                             f"decode-select (2 of them gated fallbacks) + {ndsp} decode sparse "
-                             "kernels, plus the same decode kernels replayed in a graph",
+        "gpu_launches_note": f"per step: {full_launches} full-select (1 gated re-run) + {nsp} "
+                             f"sparse + {dsel_launches} decode-select (2 of them gated "
+                             f"fallbacks) + {ndsp} decode sparse + 1 overlap kernels, plus the "
+                             "same decode kernels replayed in a graph",
         "wall_s_timed_region": round(wall, 3),
     }
 

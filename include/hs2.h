@@ -165,6 +165,31 @@ hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const
                              const int32_t* lengths, const int32_t* idx, void* o,
                              hs2_stream_t stream);
 
+/*
+ * Cross-layer selection overlap: how far two selections of the same shape
+ * pick the same global tokens.  The IndexCache page (Appendix A,
+ * "Cross-Layer Top-(k) Index Overlap") compares layers by |T(i) ∩ T(j)| / k of
+ * their top-k sets; here T is the set of global picks of a query row, the
+ * entries s of its idx row with 0 <= s <= t - W (window entries and -1
+ * padding are not part of it).  Typical use: idx_a = the selection a sparse
+ * layer inherits from its full layer, idx_b = the exact selection that layer's
+ * own queries give (hs2_full_attn_select with them).
+ *   shape                 B, L, W, k of both idx tensors (Hq, d, scale are
+ *                         checked as for the other prefill calls but unused);
+ *                         L < 2^21 - 1
+ *   idx_a, idx_b [B, L, W+k] int32   selections in the hs2_full_attn_select
+ *                         format (any slot order); entries outside [-1, t]
+ *                         are skipped and flagged as HS2_ERR_DEVICE_DATA
+ *   inter [B, L] int32    out: |T_a(t) ∩ T_b(t)| (may be NULL)
+ *   ratio [B, L] fp32     out: inter / min(k, t - W + 1); 1 for rows without
+ *                         global candidates (t < W or k = 0) (may be NULL)
+ * At least one of inter, ratio must be given.  Exact integer counting: the
+ * ratio is one correctly rounded fp32 division.
+ */
+hs2_status hs2_selection_overlap(const hs2_prefill_shape* shape, const int32_t* idx_a,
+                                 const int32_t* idx_b, int32_t* inter, float* ratio,
+                                 hs2_stream_t stream);
+
 /* Size of the fixed device scratch used by hs2_decode_select_noalloc. */
 #define HS2_NOALLOC_SCRATCH_BYTES (96u << 20)
 

@@ -191,3 +191,32 @@ def decode_sparse(q, k_cache, v_cache, idx, kv="e4m3", k_scale=None, v_scale=Non
     if rc != 0:
         raise RuntimeError(f"hs2o_decode_sparse failed ({rc})")
     return o
+
+
+def global_picks(row, t: int, W: int) -> set:
+    """The global picks of one idx row of query position t: its entries s with
+    0 <= s <= t - W (window entries and -1 padding excluded)."""
+    return {int(s) for s in row if 0 <= int(s) <= t - W}
+
+
+def selection_overlap(idx_a, idx_b, W: int, k_top: int):
+    """Cross-layer overlap of two selections [B, L, S] (the IndexCache page,
+    Appendix A, "Cross-Layer Top-(k) Index Overlap": |T(i) ∩ T(j)| / k).
+
+    Per query row t: inter = |G_a(t) ∩ G_b(t)| with G the global picks, and
+    ratio = inter / min(k, t - W + 1); rows without global candidates
+    (t < W or k = 0) get ratio 1.  Returns (inter int64 [B, L], ratio float64
+    [B, L]); plain Python sets, one row at a time."""
+    a = _np(idx_a, np.int32)
+    b = _np(idx_b, np.int32)
+    B, L, _ = a.shape
+    inter = np.zeros((B, L), dtype=np.int64)
+    ratio = np.ones((B, L), dtype=np.float64)
+    for bb in range(B):
+        for t in range(L):
+            n = len(global_picks(a[bb, t], t, W) & global_picks(b[bb, t], t, W))
+            inter[bb, t] = n
+            denom = min(k_top, t - W + 1) if (t >= W and k_top > 0) else 0
+            if denom > 0:
+                ratio[bb, t] = n / denom
+    return inter, ratio

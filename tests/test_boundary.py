@@ -131,6 +131,20 @@ def test_decode_rejects_bad_arguments(lib):
              None) == hs2.HS2_ERR_INVALID_ARG
 
 
+def test_overlap_rejects_bad_arguments(lib):
+    s = hs2.prefill_shape(1, 64, 16, 128, 8, 8)
+    f = lib.hs2_selection_overlap
+    # both outputs missing, an input missing, a misaligned output
+    assert f(ctypes.byref(s), FAKE, FAKE, None, None, None) == hs2.HS2_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), None, FAKE, FAKE, FAKE, None) == hs2.HS2_ERR_INVALID_ARG
+    assert f(ctypes.byref(s), FAKE, FAKE, FAKE + 4, None, None) == hs2.HS2_ERR_INVALID_ARG
+    # positions must fit the 21-bit hash-set entries
+    big = hs2.prefill_shape(1, (1 << 21) - 1, 16, 128, 8, 8)
+    assert f(ctypes.byref(big), FAKE, FAKE, FAKE, FAKE, None) == hs2.HS2_ERR_UNSUPPORTED
+    s_bad = hs2.prefill_shape(1, 64, 16, 128, 1024, 1025)  # W + k > 2048
+    assert f(ctypes.byref(s_bad), FAKE, FAKE, FAKE, FAKE, None) == hs2.HS2_ERR_UNSUPPORTED
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     saved = hs2._lib
     hs2._lib = None

@@ -322,3 +322,78 @@ def test_decode_needles_recovered(cuda_lib):
     _, _, idx = run_decode(cuda_lib, x)
     for b in range(4):
         assert set(x.needle_pos[b].tolist()) <= set(idx[b].tolist())
+
+
+# ------------------------------------------------- cross-layer overlap
+def _check_overlap(hs2, idx_a, idx_b, W, k, rows=None):
+    """Counts bit-exact against the oracle; ratios equal to the one correctly
+    rounded fp32 division of the exact count.  rows: flattened b*L+t sample."""
+    inter, ratio = hs2.hs2_selection_overlap(cuda(idx_a), cuda(idx_b), W, k)
+    torch.cuda.synchronize()
+    err = hs2.hs2_get_last_device_error()
+    B, L, S = idx_a.shape
+    inter = inter.cpu().numpy().reshape(-1)
+    ratio = ratio.cpu().numpy().reshape(-1)
+    if rows is None:
+        rows = np.arange(B * L)
+    ra = idx_a.reshape(B * L, 1, S)[rows]
+    rb = idx_b.reshape(B * L, 1, S)[rows]
+    oi, orat = [], []
+    for n, r in enumerate(rows):
+        t = int(r % L)
+        ga = oracle.global_picks(ra[n, 0].tolist(), t, W)
+        gb = oracle.global_picks(rb[n, 0].tolist(), t, W)
+        oi.append(len(ga & gb))
+    oi = np.array(oi)
+    assert np.array_equal(inter[rows], oi)
+    t = rows % L
+    denom = np.where((t >= W) & (k > 0), np.minimum(k, t - W + 1), 0)
+    want = np.where(denom > 0, oi.astype(np.float32) / np.maximum(denom, 1).astype(np.float32),
+                    np.float32(1.0)).astype(np.float32)
+    assert np.array_equal(ratio[rows], want)
+    return err, ratio[rows]
+
+
+@pytest.mark.parametrize("B,L,W,k", [(2, 777, 128, 256), (1, 300, 16, 0), (1, 5, 4, 8),
+                                     (3, 1500, 32, 1024), (1, 2999, 7, 30),
+                                     (1, 140000, 8, 16)])  # L > 2^17: the hash-set kernel
+def test_selection_overlap_matches_oracle(cuda_lib, B, L, W, k):
+    a, b = inputs.make_selection_pair(B, L, W, k, seed=11)
+    err, ratio = _check_overlap(cuda_lib, a, b, W, k)
+    assert err == 0
+    if k == 0:
+        assert np.all(ratio == 1.0)
+    # a selection against itself
+    err, ratio = _check_overlap(cuda_lib, a, a, W, k)
+    assert err == 0 and np.all(ratio == 1.0)
+
+
+def test_selection_overlap_of_two_layers(cuda_lib):
+    # the full layer's selection against the exact one of a sparse layer's
+    # own queries: the oracle's selections, compared on the GPU
+    x = inputs.make_workload("prefill_tiny_1k")
+    L = x.q.shape[1]
+    ia = torch.from_numpy(oracle.full_select(x.q, x.k_, x.v, x.W, x.k)["idx"]).view(1, L, -1)
+    ib = torch.from_numpy(oracle.full_select(x.q_sparse[0], x.k_, x.v, x.W, x.k)["idx"])
+    err, ratio = _check_overlap(cuda_lib, ia, ib.view(1, L, -1), x.W, x.k)
+    assert err == 0 and 0.0 < ratio.mean() < 1.0
+
+
+def test_selection_overlap_bench_size_sampled(cuda_lib):
+    # 128k rows of W=128, k=1024: every count on the GPU, 2048 rows re-counted
+    a, b = inputs.make_selection_pair(1, 131072, 128, 1024, seed=12)
+    rows = np.unique(np.concatenate([np.arange(64), np.arange(131072 - 64, 131072),
+                                     np.random.default_rng(1).choice(131072, 1920, False)]))
+    err, _ = _check_overlap(cuda_lib, a, b, 128, 1024, rows=rows)
+    assert err == 0
+
+
+def test_selection_overlap_flags_out_of_range_entries(cuda_lib):
+    a, b = inputs.make_selection_pair(1, 200, 8, 16, seed=13)
+    a = a.clone()
+    a[0, 50, 0] = 51          # beyond t = 50: skipped, flagged
+    b = b.clone()
+    b[0, 60, 3] = -7
+    err, _ = _check_overlap(cuda_lib, a, b, 8, 16)
+    assert err == cuda_lib.HS2_ERR_DEVICE_DATA
+    assert cuda_lib.hs2_get_last_device_error() == 0

@@ -365,3 +365,87 @@ def test_planted_needles_are_selected():
                              k_scale=x.k_scale, v_scale=x.v_scale)
     for b in range(B):
         assert set(x.needle_pos[b].tolist()) <= set(r["idx"][b].tolist())
+
+
+# ---------------------------------------------------------------- overlap
+# Cross-layer overlap |T(i) ∩ T(j)| / k of the IndexCache page (Appendix A),
+# applied to the global picks of HySparse2 selections.
+
+def test_overlap_hand_worked_rows():
+    # W = 2, k = 3, L = 6.  Row t: window t-1..t, candidates 0..t-2.
+    W, K, L = 2, 3, 6
+    a = -np.ones((1, L, W + K), dtype=np.int32)
+    b = -np.ones((1, L, W + K), dtype=np.int32)
+    a[0, 1, :2] = [0, 1]                 # t=1: window only -> ratio 1
+    b[0, 1, :2] = [1, 0]
+    a[0, 2, :3] = [1, 2, 0]              # t=2: one candidate, both take it -> 1/1
+    b[0, 2, :3] = [0, 1, 2]
+    a[0, 3, :4] = [2, 3, 0, 1]           # t=3: a takes {0,1}, b takes {1} of 2 -> 1/2
+    b[0, 3, :4] = [2, 3, 1, -1]
+    a[0, 5, :] = [4, 5, 3, 1, 0]         # t=5: {0,1,3} vs {1,2,3} -> 2/3
+    b[0, 5, :] = [2, 1, 4, 3, 5]
+    inter, ratio = oracle.selection_overlap(a, b, W, K)
+    assert inter[0].tolist() == [0, 0, 1, 1, 0, 2]
+    # t=0: no candidates; t=4: both empty of 3 candidates -> 0/3
+    assert ratio[0].tolist() == [1.0, 1.0, 1.0, 0.5, 0.0, 2.0 / 3.0]
+
+
+def test_overlap_against_brute_force_pair_count():
+    rng = np.random.default_rng(7)
+    W, K, L, B = 4, 16, 200, 2
+    a = -np.ones((B, L, W + K), dtype=np.int32)
+    b = -np.ones((B, L, W + K), dtype=np.int32)
+    for bb in range(B):
+        for t in range(L):
+            n = min(t + 1, W + K)
+            for arr in (a, b):
+                picks = rng.choice(t + 1, size=n, replace=False)
+                arr[bb, t, :n] = picks
+    inter, ratio = oracle.selection_overlap(a, b, W, K)
+    for bb in range(B):
+        for t in range(L):
+            # every (i, j) pair of global entries, counted with plain loops
+            cnt = 0
+            for x in a[bb, t]:
+                for y in b[bb, t]:
+                    if x == y and 0 <= x <= t - W:
+                        cnt += 1
+            assert inter[bb, t] == cnt
+            if t >= W:
+                assert ratio[bb, t] == cnt / min(K, t - W + 1)
+
+
+def test_overlap_of_real_selections_matches_numpy_intersect():
+    x = inputs.make_workload("prefill_tiny_1k")
+    q2 = x.q_sparse[0]
+    L = x.q.shape[1]
+    idx_a = oracle.full_select(x.q, x.k_, x.v, x.W, x.k)["idx"].reshape(1, L, -1)
+    idx_b = oracle.full_select(q2, x.k_, x.v, x.W, x.k)["idx"].reshape(1, L, -1)
+    inter, ratio = oracle.selection_overlap(idx_a, idx_b, x.W, x.k)
+    a, b = np.asarray(idx_a), np.asarray(idx_b)
+    for t in range(L):
+        ga = a[0, t][(a[0, t] >= 0) & (a[0, t] <= t - x.W)]
+        gb = b[0, t][(b[0, t] >= 0) & (b[0, t] <= t - x.W)]
+        assert inter[0, t] == np.intersect1d(ga, gb).size
+    # a selection against itself: every row overlaps fully
+    same_i, same_r = oracle.selection_overlap(idx_a, idx_a, x.W, x.k)
+    assert np.all(same_r == 1.0)
+    # a query with itself agrees; a fresh query mostly does not repeat the picks
+    assert 0.0 <= ratio.mean() < 1.0
+
+
+def test_overlap_ignores_slot_order_window_and_padding():
+    rng = np.random.default_rng(3)
+    W, K, L = 3, 5, 40
+    a = -np.ones((1, L, W + K), dtype=np.int32)
+    b = -np.ones((1, L, W + K), dtype=np.int32)
+    for t in range(L):
+        n = min(t + 1, W + K)
+        a[0, t, :n] = rng.choice(t + 1, size=n, replace=False)
+        b[0, t, :n] = rng.choice(t + 1, size=n, replace=False)
+    i0, r0 = oracle.selection_overlap(a, b, W, K)
+    a2 = a.copy()
+    for t in range(L):
+        a2[0, t] = rng.permutation(a2[0, t])
+    i1, r1 = oracle.selection_overlap(a2, b, W, K)
+    assert np.array_equal(i0, i1) and np.array_equal(r0, r1)

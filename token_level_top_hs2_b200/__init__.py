@@ -37,7 +37,7 @@ EXPORTED = [
     "hs2_status_string", "hs2_version", "hs2_full_attn_select_workspace",
     "hs2_full_attn_select", "hs2_sparse_attn", "hs2_decode_select_workspace",
     "hs2_decode_select", "hs2_decode_sparse", "hs2_get_last_device_error",
-    "hs2_decode_select_noalloc",
+    "hs2_decode_select_noalloc", "hs2_selection_overlap",
 ]
 
 
@@ -91,6 +91,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_decode_sparse.restype = i32
     L.hs2_decode_select_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.hs2_decode_select_noalloc.restype = i32
+    L.hs2_selection_overlap.argtypes = [P, vp, vp, vp, vp, vp]
+    L.hs2_selection_overlap.restype = i32
     L.hs2_get_last_device_error.argtypes = [vp]
     L.hs2_get_last_device_error.restype = i32
     _lib = L
@@ -219,6 +221,23 @@ def hs2_decode_sparse(q, k_cache, v_cache, lengths, idx, *, kv="e4m3", k_scale=N
                                   _ptr(lengths), _ptr(idx), _ptr(o), _stream(stream))
     _check(st, "hs2_decode_sparse")
     return o
+
+
+def hs2_selection_overlap(idx_a, idx_b, W: int, k_top: int, *, inter=None, ratio=None,
+                          stream=None):
+    """idx_a, idx_b [B,L,W+k] int32 selections. Returns (inter [B,L] int32, ratio [B,L] fp32):
+    per query row the number of global picks the two share and that number over
+    min(k, t-W+1)."""
+    B, L, S = idx_a.shape
+    # head count, head dim and scale do not enter the overlap; any valid values do
+    shape = prefill_shape(B, L, 16, 128, W, k_top)
+    dev = idx_a.device
+    inter = torch.empty(B, L, dtype=torch.int32, device=dev) if inter is None else inter
+    ratio = torch.empty(B, L, dtype=torch.float32, device=dev) if ratio is None else ratio
+    st = load().hs2_selection_overlap(ctypes.byref(shape), _ptr(idx_a), _ptr(idx_b), _ptr(inter),
+                                      _ptr(ratio), _stream(stream))
+    _check(st, "hs2_selection_overlap")
+    return inter, ratio
 
 
 def hs2_get_last_device_error(stream=None) -> int:

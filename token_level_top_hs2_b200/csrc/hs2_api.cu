@@ -7,6 +7,7 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/hs2.h"
@@ -15,6 +16,7 @@
 #include "decode_pass1.cuh"
 #include "decode_sketch.cuh"
 #include "decode_tc.cuh"
+#include "overlap.cuh"
 #include "prefill_kernels.cuh"
 #include "prefill_tc.cuh"
 #include "sparse_kernels.cuh"
@@ -703,6 +705,39 @@ hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const
                                              lengths, idx, o, st, flags);
     return run_decode_sparse<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths,
                                         idx, o, st, flags);
+}
+
+hs2_status hs2_selection_overlap(const hs2_prefill_shape* shape, const int32_t* idx_a,
+                                 const int32_t* idx_b, int32_t* inter, float* ratio,
+                                 hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (!idx_a || !idx_b || (!inter && !ratio)) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(idx_a) || !aligned16(idx_b) || (inter && !aligned16(inter)) ||
+        (ratio && !aligned16(ratio)))
+        return HS2_ERR_INVALID_ARG;
+    if (shape->L >= (1 << ovl::kPosBits) - 1) return HS2_ERR_UNSUPPORTED;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long rows = (long long)shape->B * shape->L;
+    const bool use_bitmap = shape->L <= ovl::kBitmapMaxL;
+    auto kern = use_bitmap ? ovl::overlap_bitmap_kernel : ovl::overlap_kernel;
+    const size_t smem = use_bitmap ? ovl::bitmap_smem_bytes(shape->W + shape->k, shape->L)
+                                   : ovl::smem_bytes(shape->W + shape->k, shape->k);
+    if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+    // per warp a bitmap (or hash set) and two stages of both rows; each warp
+    // walks many rows
+    const size_t per_sm_smem = 228 * 1024;  // shared memory of one SM (1 KB per CTA reserved)
+    const long long per_sm = std::max<long long>(1, (long long)(per_sm_smem / (smem + 1024)));
+    const long long want = (rows + ovl::kWarps - 1) / ovl::kWarps;
+    const int grid = (int)std::min<long long>(want, per_sm * sms);
+    kern<<<grid, ovl::kWarps * 32, smem, st>>>(idx_a, idx_b, shape->B, shape->L, shape->W + shape->k,
+                                               shape->W, shape->k, inter, ratio, flags);
+    return launch_status();
 }
 
 hs2_status hs2_get_last_device_error(hs2_stream_t stream) {

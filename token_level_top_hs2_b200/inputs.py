@@ -194,3 +194,42 @@ def make_workload(name: str, repeat: int = 0):
     if kind == "prefill":
         return make_prefill(seed=seed, **w)
     return make_decode(seed=seed, **w)
+
+
+def make_selection_pair(B: int, L: int, W: int, k: int, *, seed: int, shuffle: bool = True):
+    """Two synthetic selections [B, L, W+k] int32 in the library's idx format,
+    for overlap checks.  Row t: the window max(0, t-W+1)..t, then min(k, n)
+    distinct global picks from the n = t-W+1 candidates, then -1 padding.
+    The picks of the first selection are (a*j + c) mod n for j < min(k, n),
+    with a random multiplier a coprime to n; the second uses the same a and
+    c + s for a random shift s in [0, k], so rows overlap by every amount
+    from all to nothing.  With shuffle, each row's slots are permuted."""
+    g = torch.Generator().manual_seed(seed)
+    S = W + k
+    t = torch.arange(L, dtype=torch.int64).view(1, L, 1).expand(B, L, 1)
+    n = (t - W + 1).clamp(min=0)                                   # candidates per row
+    primes = torch.tensor([1000003, 999983, 999979, 999961, 999959, 999953], dtype=torch.int64)
+    a = primes[torch.randint(0, len(primes), (B, L, 1), generator=g)]
+    nn = n.clamp(min=1)
+    a = torch.where(torch.gcd(a, nn) == 1, a, torch.ones_like(a))  # coprime: distinct picks
+    c = torch.randint(0, 1 << 30, (B, L, 1), generator=g)
+    s = torch.randint(0, k + 1, (B, L, 1), generator=g)
+    j = torch.arange(k, dtype=torch.int64).view(1, 1, k)
+    used = j < n                                                     # min(k, n) picks
+    ga = torch.where(used, (a * j + c) % nn, torch.full_like(j, -1))
+    gb = torch.where(used, (a * j + c + s) % nn, torch.full_like(j, -1))
+    w = torch.arange(W, dtype=torch.int64).view(1, 1, W)
+    win = t - W + 1 + w
+    win = torch.where(win >= 0, win, torch.full_like(win, -1))
+    out = []
+    for glob in (ga, gb):
+        row = torch.cat([win, glob], dim=2)
+        # valid entries first (window, then globals), -1 padding at the tail
+        key = torch.where(row >= 0, torch.zeros_like(row), torch.ones_like(row))
+        order = torch.argsort(key * (2 * S) + torch.arange(S).view(1, 1, S), dim=2)
+        row = torch.gather(row, 2, order)
+        if shuffle:
+            perm = torch.argsort(torch.rand(B, L, S, generator=g), dim=2)
+            row = torch.gather(row, 2, perm)
+        out.append(row.to(torch.int32).contiguous())
+    return out[0], out[1]
