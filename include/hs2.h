@@ -114,6 +114,30 @@ hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, c
                                 void* workspace, size_t workspace_bytes, hs2_stream_t stream);
 
 /*
+ * Block-level selector variant: the full layer of HySparse, the predecessor
+ * the HySparse2 summary compares against ("Limits": 64-token blocks, 1,024
+ * global tokens, a separate 128-token local window).  Same exact attention
+ * (o, lse) as hs2_full_attn_select; the selection takes whole blocks:
+ *   - blocks are the aligned `block`-token ranges [block*j, block*j+block-1];
+ *   - a block is a candidate if it holds a position <= t - W; its attention
+ *     mass is the sum of score(t,s) over its positions s <= t - W (the
+ *     head-summed probability, as for the token selector);
+ *   - the k / block candidate blocks of largest mass are chosen, ties to the
+ *     lower block, all of them when there are at most k / block;
+ *   - idx row: the window ascending, then the positions <= t - W of the chosen
+ *     blocks (ascending block order), then -1.  Same [B, L, W+k] format, so
+ *     hs2_sparse_attn consumes it unchanged.
+ * block must be 64; k a positive multiple of it.  The workspace holds the lse
+ * (when lse is NULL) and one fp32 mass per (row, block): 4 * B * L * ceil(L/64)
+ * bytes, 1 GiB at L = 128k.
+ */
+size_t hs2_full_attn_select_blocks_workspace(const hs2_prefill_shape* shape, int block);
+hs2_status hs2_full_attn_select_blocks(const hs2_prefill_shape* shape, int block, const void* q,
+                                       const void* k, const void* v, void* o, float* lse,
+                                       int32_t* idx, void* workspace, size_t workspace_bytes,
+                                       hs2_stream_t stream);
+
+/*
  * Sparse layer (prefill): each query token attends, with its own queries, only
  * to the K/V rows its inherited index set names (KV Reuse, "How it works").
  *   q   [B, L, Hq, d] bf16      this sparse layer's queries

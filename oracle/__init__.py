@@ -220,3 +220,42 @@ def selection_overlap(idx_a, idx_b, W: int, k_top: int):
             if denom > 0:
                 ratio[bb, t] = n / denom
     return inter, ratio
+
+
+def block_select(q, k, v, W: int, k_top: int, block: int = 64, rows=None, scale=None):
+    """Block-level selector of HySparse (64-token blocks, the same forced
+    window), from the oracle's fp64 score rows.
+
+    Candidate blocks of row t: the aligned `block`-position ranges that hold a
+    position <= t - W; mass(t, j) = sum of score(t, s) over the block's
+    positions s <= t - W.  The k_top/block blocks of largest mass are chosen
+    (ties to the lower block; all when there are fewer).  Returns dict:
+    idx [R, W+k] (window ascending, then the chosen blocks' candidate positions
+    in ascending block order, -1 padding), mass [R, nblk] (0 beyond the
+    candidates), sigma [R] (the smallest chosen mass, -1 when every block is
+    taken), rows."""
+    B, L = q.shape[:2]
+    out = full_select(q, k, v, W, k_top, rows=rows, scale=scale, want_score_row=True)
+    sr, rows = out["score_row"], out["rows"]
+    R, S = rows.shape[0], W + k_top
+    nsel = k_top // block
+    nblk = (L + block - 1) // block
+    idx = -np.ones((R, S), dtype=np.int32)
+    mass = np.zeros((R, nblk))
+    sigma = -np.ones(R)
+    for r in range(R):
+        t = int(rows[r] % L)
+        w0 = max(0, t - W + 1)
+        win = list(range(w0, t + 1))
+        last = t - W
+        nb = last // block + 1 if last >= 0 else 0
+        for j in range(nb):
+            mass[r, j] = float(np.sum(sr[r, block * j: min(block * j + block, last + 1)]))
+        order = sorted(range(nb), key=lambda j: (-mass[r, j], j))
+        chosen = sorted(order[:nsel])
+        if nb > nsel:
+            sigma[r] = mass[r, order[nsel - 1]]
+        glob = [s for j in chosen for s in range(block * j, min(block * j + block, last + 1))]
+        row = win + glob
+        idx[r, :len(row)] = row
+    return dict(idx=idx, mass=mass, sigma=sigma, rows=rows)

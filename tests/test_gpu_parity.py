@@ -397,3 +397,63 @@ def test_selection_overlap_flags_out_of_range_entries(cuda_lib):
     err, _ = _check_overlap(cuda_lib, a, b, 8, 16)
     assert err == cuda_lib.HS2_ERR_DEVICE_DATA
     assert cuda_lib.hs2_get_last_device_error() == 0
+
+
+# ------------------------------------------------- block-level selector
+def _check_block_rows(idx, ora, rows, L, W, k, blk):
+    """Windows identical; chosen blocks equal to the oracle's except swaps whose
+    oracle mass lies within 1e-5 (relative) of the smallest chosen mass; every
+    chosen block contributes exactly its candidate positions."""
+    n_swap = 0
+    for r, row in enumerate(rows):
+        t = int(row % L)
+        g = idx[row]
+        o = ora["idx"][r]
+        wl = min(t + 1, W)
+        assert g[:wl].tolist() == o[:wl].tolist(), t
+        gg = g[wl:][g[wl:] >= 0]
+        og = o[wl:][o[wl:] >= 0]
+        gb, ob = set((gg // blk).tolist()), set((og // blk).tolist())
+        assert len(gb) == len(ob) and len(gg) == len(set(gg.tolist()))
+        for j in gb:
+            want = list(range(blk * j, min(blk * j + blk, t - W + 1)))
+            assert sorted(s for s in gg.tolist() if s // blk == j) == want, (t, j)
+        diff = gb ^ ob
+        if diff:
+            sig = ora["sigma"][r]
+            assert sig > 0
+            for j in diff:
+                assert abs(ora["mass"][r, j] - sig) <= 1e-5 * sig, (t, j)
+            n_swap += len(diff) // 2
+        assert np.all(g[wl + len(gg):] == -1)
+    return n_swap
+
+
+@pytest.mark.parametrize("shape", [
+    dict(B=1, L=1024, Hq=4, d=64, W=32, k=128, n_topics=8, seg=128),
+    dict(B=2, L=777, Hq=16, d=128, W=128, k=256, n_topics=8, seg=256),
+    dict(B=1, L=5, Hq=16, d=64, W=4, k=64, n_topics=2, seg=4),
+    dict(B=1, L=3000, Hq=8, d=128, W=64, k=1024, n_topics=8, seg=256),
+])
+def test_block_selector_matches_oracle(cuda_lib, shape):
+    s = dict(shape)
+    x = inputs.make_prefill(seed=inputs.seed_for(0, 2), n_sparse=1, **s)
+    B, L, Hq, d = x.q.shape
+    o, lse, idx = cuda_lib.hs2_full_attn_select_blocks(cuda(x.q), cuda(x.k_), cuda(x.v), x.W, x.k)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    o = o.float().cpu().numpy().reshape(B * L, Hq, d)
+    lse = lse.cpu().numpy().reshape(B * L, Hq)
+    idx = idx.cpu().numpy().reshape(B * L, -1)
+    rows = np.arange(B * L) if B * L <= 1600 else sample_rows(B, L, 512, seed=3, seg=shape["seg"])
+    ora = oracle.block_select(x.q, x.k_, x.v, x.W, x.k, block=64, rows=rows)
+    full = oracle.full_select(x.q, x.k_, x.v, x.W, x.k, rows=rows)
+    assert max_abs(o[rows], full["o"]) <= TOL_BF16
+    assert max_abs(lse[rows], full["lse"]) <= TOL_LSE
+    _check_block_rows(idx, ora, rows, L, x.W, x.k, 64)
+    # the sparse layer consumes the block selection unchanged
+    idx_t = torch.from_numpy(idx).view(B, L, -1)
+    os_ = cuda_lib.hs2_sparse_attn(cuda(x.q_sparse[0]), cuda(x.k_), cuda(x.v), cuda(idx_t),
+                                  W=x.W, k_top=x.k)
+    ref = oracle.sparse(x.q_sparse[0], x.k_, x.v, idx_t, rows=rows)
+    assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d)[rows], ref) <= TOL_BF16

@@ -449,3 +449,83 @@ def test_overlap_ignores_slot_order_window_and_padding():
         a2[0, t] = rng.permutation(a2[0, t])
     i1, r1 = oracle.selection_overlap(a2, b, W, K)
     assert np.array_equal(i0, i1) and np.array_equal(r0, r1)
+
+
+# ------------------------------------------------- block-level selector
+# HySparse (the predecessor in the HySparse2 summary, "Limits"): 64-token
+# blocks ranked by attention mass (page 3's reading: the sum of the attention
+# scores inside a block), the same forced window.
+
+def _independent_block_selection(score_row, t, W, k, block):
+    """Masses as plain sums of torch float64 scores; blocks ranked by
+    (mass desc, index asc) with numpy's lexsort; positions <= t-W."""
+    w = list(range(max(0, t - W + 1), t + 1))
+    last = t - W
+    if last < 0:
+        return w, [], np.zeros(0)
+    nb = last // block + 1
+    mass = np.array([score_row[block * j: min(block * j + block, last + 1)].sum()
+                     for j in range(nb)])
+    nsel = k // block
+    if nb <= nsel:
+        chosen = list(range(nb))
+    else:
+        order = np.lexsort((np.arange(nb), -mass))
+        chosen = sorted(order[:nsel].tolist())
+    return w, [s for j in chosen for s in range(block * j, min(block * j + block, last + 1))], mass
+
+
+def test_block_selection_matches_torch_masses_and_sort():
+    B, L, Hq, d, W, k, blk = 1, 700, 4, 16, 16, 256, 64
+    x = inputs.make_prefill(B, L, Hq, d, W, k, n_topics=4, seg=32, seed=21)
+    r = oracle.block_select(x.q, x.k_, x.v, W, k, block=blk)
+    _, _, score = ref_full(x.q, x.k_, x.v, x.scale)
+    score = score.numpy()[0]
+    for t in range(L):
+        w, glob, mass = _independent_block_selection(score[t], t, W, k, blk)
+        got = r["idx"][t]
+        got = got[got >= 0].tolist()
+        assert got == w + glob, t
+        np.testing.assert_allclose(r["mass"][t, : mass.size], mass, rtol=1e-12, atol=1e-15)
+
+
+def test_block_selection_all_keys_equal_takes_the_first_full_blocks():
+    """Uniform scores Hq/(t+1): every full candidate block has the same mass,
+    a partial last block less; ties go to the lower blocks."""
+    B, L, Hq, d, W, k, blk = 1, 600, 4, 8, 16, 128, 64
+    g = torch.Generator().manual_seed(8)
+    q = torch.randn(B, L, Hq, d, generator=g).bfloat16()
+    krow = torch.randn(d, generator=g).bfloat16()
+    kk = krow.expand(B, L, d).contiguous()
+    v = torch.randn(B, L, d, generator=g).bfloat16()
+    r = oracle.block_select(q, kk, v, W, k, block=blk)
+    for t in [16, 79, 80, 143, 144, 300, 599]:
+        last = t - W
+        nb = last // blk + 1
+        got = r["idx"][t]
+        glob = got[got >= 0].tolist()[min(t + 1, W):]
+        if nb <= k // blk:
+            assert glob == list(range(last + 1))
+        else:
+            assert glob == list(range(2 * blk))  # blocks 0 and 1
+        np.testing.assert_allclose(r["mass"][t, 0], min(blk, last + 1) * Hq / (t + 1),
+                                   rtol=1e-12)
+
+
+def test_block_selection_structure():
+    B, L, Hq, d, W, k, blk = 2, 333, 8, 32, 8, 192, 64
+    x = inputs.make_prefill(B, L, Hq, d, W, k, n_topics=4, seg=32, seed=22)
+    r = oracle.block_select(x.q, x.k_, x.v, W, k, block=blk)
+    for row in range(B * L):
+        t = row % L
+        got = r["idx"][row]
+        sel = got[got >= 0]
+        wl = min(t + 1, W)
+        assert sel[:wl].tolist() == list(range(t - wl + 1, t + 1))
+        glob = sel[wl:]
+        assert len(glob) == len(set(glob.tolist())) and np.all(glob <= t - W)
+        blocks = sorted(set((glob // blk).tolist()))
+        assert len(blocks) <= k // blk
+        for j in blocks:  # whole blocks, clipped at t-W
+            want = list(range(blk * j, min(blk * j + blk, t - W + 1)))
+            assert [s for s in glob.tolist() if s // blk == j] == want

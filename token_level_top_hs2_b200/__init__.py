@@ -38,6 +38,7 @@ EXPORTED = [
     "hs2_full_attn_select", "hs2_sparse_attn", "hs2_decode_select_workspace",
     "hs2_decode_select", "hs2_decode_sparse", "hs2_get_last_device_error",
     "hs2_decode_select_noalloc", "hs2_selection_overlap",
+    "hs2_full_attn_select_blocks_workspace", "hs2_full_attn_select_blocks",
 ]
 
 
@@ -81,6 +82,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_full_attn_select_workspace.restype = sz
     L.hs2_full_attn_select.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.hs2_full_attn_select.restype = i32
+    L.hs2_full_attn_select_blocks_workspace.argtypes = [P, i32]
+    L.hs2_full_attn_select_blocks_workspace.restype = sz
+    L.hs2_full_attn_select_blocks.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.hs2_full_attn_select_blocks.restype = i32
     L.hs2_sparse_attn.argtypes = [P, vp, vp, vp, i32, vp, vp, vp, vp, vp]
     L.hs2_sparse_attn.restype = i32
     L.hs2_decode_select_workspace.argtypes = [D]
@@ -160,6 +165,29 @@ def hs2_full_attn_select(q, k, v, W: int, k_top: int, *, scale=None, o=None, lse
                                      _ptr(lse), _ptr(idx), _ptr(workspace),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hs2_full_attn_select")
+    return o, lse, idx
+
+
+def hs2_full_attn_select_blocks(q, k, v, W: int, k_top: int, *, block: int = 64, scale=None,
+                                o=None, lse=None, idx=None, workspace=None, want_lse: bool = True,
+                                stream=None):
+    """Block-level selector variant (HySparse): as hs2_full_attn_select, with the
+    k_top global tokens taken as k_top/block whole blocks of largest attention mass."""
+    B, L, Hq, d = q.shape
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    dev = q.device
+    o = torch.empty_like(q) if o is None else o
+    if lse is None and want_lse:
+        lse = torch.empty(B, L, Hq, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, L, W + k_top, dtype=torch.int32, device=dev) if idx is None else idx
+    need = load().hs2_full_attn_select_blocks_workspace(ctypes.byref(shape), block)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    st = load().hs2_full_attn_select_blocks(ctypes.byref(shape), block, _ptr(q), _ptr(k), _ptr(v),
+                                            _ptr(o), _ptr(lse), _ptr(idx), _ptr(workspace),
+                                            workspace.numel() * workspace.element_size(),
+                                            _stream(stream))
+    _check(st, "hs2_full_attn_select_blocks")
     return o, lse, idx
 
 

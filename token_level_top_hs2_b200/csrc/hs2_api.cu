@@ -227,11 +227,27 @@ PrefillWs prefill_ws(const hs2_prefill_shape* s) {
     return w;
 }
 
+// Block-level selector workspace: lse (when the caller passes none), then the
+// attention mass of every (row, 64-key block).
+struct BlockWs {
+    size_t lse_off, mass_off, nblk, total;
+};
+BlockWs block_ws(const hs2_prefill_shape* s) {
+    BlockWs w;
+    const size_t rows = (size_t)s->B * s->L;
+    w.lse_off = 0;
+    w.nblk = (size_t)(s->L + tcfa::kBlock - 1) / tcfa::kBlock;
+    w.mass_off = round_up(rows * s->Hq * sizeof(float), 256);
+    w.total = w.mass_off + rows * w.nblk * sizeof(float);
+    return w;
+}
+
 template <int D>
 hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void* k,
                            const void* v, void* o, float* lse, int32_t* idx, uint8_t* ws,
-                           cudaStream_t st, unsigned* flags) {
+                           cudaStream_t st, unsigned* flags, bool blocks = false) {
     const PrefillWs w = prefill_ws(s);
+    const BlockWs bw = block_ws(s);  // same lse area (offset 0) as the token path
     float* lse_p = lse ? lse : reinterpret_cast<float*>(ws + w.lse_off);
     const float scale2 = s->scale * kLog2e;
     {
@@ -253,19 +269,35 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
             !map_kv(&mk, k, s->B, s->L, D, tcfa::SBN))
             return HS2_ERR_CUDA;
         const size_t smem = tcfa::Sel<D>::SMEM;
+        dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->B);
+        if (blocks) {
+            // block masses, then the choice of blocks per row
+            auto kb = tcfa::prefill_select_tc_kernel<D, true>;
+            if (!set_smem(kb, smem)) return HS2_ERR_CUDA;
+            float* mass = reinterpret_cast<float*>(ws + bw.mass_off);
+            kb<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k,
+                                                   s->W + s->k, 0, scale2, nullptr, idx, 0,
+                                                   nullptr, nullptr, flags, mass, (int)bw.nblk);
+            if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
+            const long long rows = (long long)s->B * s->L;
+            const long long want = (rows + tcfa::kBlkWarps - 1) / tcfa::kBlkWarps;
+            const int g2 = (int)std::min<long long>(want, 148LL * 16);
+            tcfa::block_select_kernel<<<g2, tcfa::kBlkWarps * 32, 0, st>>>(
+                mass, s->B, s->L, s->W, s->k / tcfa::kBlock, s->W + s->k, (int)bw.nblk, idx);
+            return launch_status();
+        }
         auto kern = tcfa::prefill_select_tc_kernel<D>;
         if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
-        dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->B);
         unsigned* fail = reinterpret_cast<unsigned*>(ws + w.fail_off);
         uint64_t* buf = reinterpret_cast<uint64_t*>(ws + w.buf_off);
         if (cudaMemsetAsync(fail, 0, w.fail_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
         // speculative thresholds, then the exact selection for the query blocks
         // whose rows failed the check (a gated launch: the others return at once)
         kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
-                                      pf_cap(s->k), scale2, buf, idx, 1, nullptr, fail, flags);
+                                      pf_cap(s->k), scale2, buf, idx, 1, nullptr, fail, flags, nullptr, 0);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
         kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
-                                      pf_cap(s->k), scale2, buf, idx, 0, fail, nullptr, flags);
+                                      pf_cap(s->k), scale2, buf, idx, 0, fail, nullptr, flags, nullptr, 0);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     return HS2_OK;
@@ -623,6 +655,34 @@ hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, c
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (shape->d == 128) return run_full_select<128>(shape, q, k, v, o, lse, idx, ws, st, flags);
     return run_full_select<64>(shape, q, k, v, o, lse, idx, ws, st, flags);
+}
+
+size_t hs2_full_attn_select_blocks_workspace(const hs2_prefill_shape* shape, int block) {
+    if (check_prefill(shape) != HS2_OK || block != tcfa::kBlock) return 0;
+    return block_ws(shape).total;
+}
+
+hs2_status hs2_full_attn_select_blocks(const hs2_prefill_shape* shape, int block, const void* q,
+                                       const void* k, const void* v, void* o, float* lse,
+                                       int32_t* idx, void* workspace, size_t workspace_bytes,
+                                       hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (block != tcfa::kBlock) return HS2_ERR_UNSUPPORTED;
+    if (shape->k < block || shape->k % block != 0) return HS2_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !idx || !workspace) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(idx) ||
+        !aligned16(workspace) || (lse && !aligned16(lse)))
+        return HS2_ERR_INVALID_ARG;
+    if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
+    if (workspace_bytes < block_ws(shape).total) return HS2_ERR_WORKSPACE;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    if (shape->d == 128)
+        return run_full_select<128>(shape, q, k, v, o, lse, idx, ws, st, flags, true);
+    return run_full_select<64>(shape, q, k, v, o, lse, idx, ws, st, flags, true);
 }
 
 hs2_status hs2_sparse_attn(const hs2_prefill_shape* shape, const void* q, const void* k,

@@ -472,7 +472,12 @@ HS2_DEV uint64_t warp_cut(uint64_t* buf, int cnt, int k, int* hist) {
 }
 
 // grid (ceil(L/128), B), 320 threads.  wsbuf: [B*L][2][cap] keys.
-template <int D>
+// BLK (the block-level selector of HySparse, the predecessor the HySparse2
+// summary ablates against in "Limits"): instead of streaming token
+// candidates, every score thread writes the attention mass of the 64-key
+// blocks it holds -- the sum of its candidates' scores -- to
+// mass[b*L + t][nblk]; block_select_kernel picks the blocks.
+template <int D, bool BLK = false>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                          const __grid_constant__ CUtensorMap map_k,
@@ -480,7 +485,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                          int cap, float scale2, uint64_t* __restrict__ wsbuf,
                          int32_t* __restrict__ idx, int speculate,
                          const unsigned* __restrict__ gate, unsigned* __restrict__ fail_qb,
-                         unsigned* __restrict__ flags) {
+                         unsigned* __restrict__ flags, float* __restrict__ mass, int nblk) {
     using F = Sel<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -615,7 +620,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         for (int kb = 0; kb < n_kb && ok; kb++) {
             const int key0 = kb * SBN + half * 128;
             const bool streams = valid && key0 <= maxkey;
-            {
+            if constexpr (!BLK) {
                 // make room for this block's 128 candidates before accumulating
                 unsigned need = __ballot_sync(0xffffffffu, streams && cnt + 128 > cap);
                 while (need) {
@@ -678,6 +683,32 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 if (lane == 0) mbar_arrive(&bars.s_empty[buf]);
             }
             if (!ok) break;
+            if constexpr (BLK) {
+                // ---- all heads summed: the mass of each 64-key block with a
+                // candidate (eight partial sums of eight, then a tree)
+                if (streams) {
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        const int bk0 = key0 + 64 * u;
+                        if (bk0 > maxkey) break;
+                        float p8[8];
+#pragma unroll
+                        for (int g = 0; g < 8; g++) {
+                            float a = 0.f;
+#pragma unroll
+                            for (int i = 0; i < 8; i++) {
+                                const int j = 64 * u + 8 * g + i;
+                                a += (key0 + j <= maxkey) ? acc[j] : 0.f;
+                            }
+                            p8[g] = a;
+                        }
+                        const float m = ((p8[0] + p8[1]) + (p8[2] + p8[3])) +
+                                        ((p8[4] + p8[5]) + (p8[6] + p8[7]));
+                        mass[((size_t)b * L + t) * nblk + bk0 / 64] = m;
+                    }
+                }
+                continue;
+            }
             // ---- all heads summed: stream the block's candidates
             if (streams) {
 #pragma unroll
@@ -702,6 +733,13 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     }
     fence_before_sync();
     __syncthreads();
+    if constexpr (BLK) {
+        if (warp == 0) {
+            fence_after_sync();
+            tmem_dealloc(tmem, 512);
+        }
+        return;
+    }
     // ---------------------------------------------- final selection per row
     // Warps 2..9: warp w takes rows w-2, w+6, ... (16 rows each).  The union of
     // a row's two streams is histogrammed relative to the higher stream
@@ -832,6 +870,81 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
     if (warp == 0) {
         fence_after_sync();
         tmem_dealloc(tmem, 512);
+    }
+}
+
+// Block-level selection (HySparse's selector: 64-token blocks, the same
+// forced window).  One warp per query row t: the candidate blocks are the
+// aligned 64-key blocks with a position <= t - W; the nsel = k / 64 blocks of
+// largest attention mass are taken (ties to the lower block; all of them when
+// there are at most nsel), and the row gets the window ascending, then the
+// candidate positions of the chosen blocks (in block order), then -1.
+constexpr int kBlkWarps = 4;
+constexpr int kBlock = 64;
+
+__global__ void __launch_bounds__(kBlkWarps * 32)
+block_select_kernel(const float* __restrict__ mass, int B, int L, int W, int nsel, int S,
+                    int nblk, int32_t* __restrict__ idx) {
+    __shared__ int hist_all[kBlkWarps][256];
+    __shared__ int sel_all[kBlkWarps][64];   // chosen blocks, ascending
+    __shared__ int off_all[kBlkWarps][65];   // output offset of each chosen block
+    const int warp = threadIdx.x >> 5, lane = lane_id();
+    int* hist = hist_all[warp];
+    int* sel = sel_all[warp];
+    int* off = off_all[warp];
+    const long long rows = (long long)B * L;
+    for (long long r = (long long)blockIdx.x * kBlkWarps + warp; r < rows;
+         r += (long long)gridDim.x * kBlkWarps) {
+        const int t = (int)(r % L);
+        int32_t* out = idx + r * S;
+        const int w0 = max(0, t - W + 1);
+        const int wl = t - w0 + 1;
+        for (int i = lane; i < wl; i += 32) out[i] = w0 + i;
+        const int last = t - W;  // candidates 0..last
+        const int nb = last >= 0 ? last / kBlock + 1 : 0;
+        const float* mrow = mass + r * nblk;
+        // key = mass bits << 32 | ~block: larger is better, ties to the lower block
+        auto key = [&](int i) {
+            return ((uint64_t)__float_as_uint(__ldg(mrow + i)) << 32) | (uint64_t)(~(uint32_t)i);
+        };
+        const uint64_t thr = (nb > nsel) ? warp_radix_threshold(key, nb, nsel, hist) : 0ull;
+        // the chosen blocks in ascending order, and their output offsets
+        int n_sel = 0, total = 0;
+        for (int i0 = 0; i0 < nb; i0 += 32) {
+            const int i = i0 + lane;
+            const bool take = i < nb && (nb <= nsel || key(i) >= thr);
+            const unsigned bal = __ballot_sync(0xffffffffu, take);
+            const int cnt = take ? min(kBlock, last - kBlock * i + 1) : 0;
+            // inclusive scan of the token counts over the lanes
+            int inc = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, inc, o);
+                if (lane >= o) inc += v;
+            }
+            if (take) {
+                const int p = n_sel + __popc(bal & ((1u << lane) - 1));
+                sel[p] = i;
+                off[p] = total + inc - cnt;
+            }
+            n_sel += __popc(bal);
+            total += __shfl_sync(0xffffffffu, inc, 31);
+        }
+        __syncwarp();
+        if (lane == 0) off[n_sel] = total;
+        __syncwarp();
+        // write the chosen positions: entry e belongs to the block whose offset
+        // range holds it
+        for (int e = lane; e < total; e += 32) {
+            int lo = 0, hi = n_sel - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (off[mid] <= e) lo = mid; else hi = mid - 1;
+            }
+            out[wl + e] = kBlock * sel[lo] + (e - off[lo]);
+        }
+        for (int i = wl + total + lane; i < S; i += 32) out[i] = -1;
+        __syncwarp();
     }
 }
 
