@@ -252,6 +252,14 @@ def run_ours(args, world, rank, local):
     def overlap():
         hs2.hs2_selection_overlap(idx, idx_own, W, K, inter=inter, ratio=ratio)
 
+    # HySparse's block-level selector on the same layer (64-token blocks)
+    bws = torch.empty(hs2.hs2_full_attn_select_blocks_workspace(
+        hs2.prefill_shape(B, L, Hq, d, W, K), 64), dtype=torch.uint8, device=dev)
+    bidx = torch.empty_like(idx)
+
+    def full_blocks():
+        hs2.hs2_full_attn_select_blocks(q, k, v, W, K, o=o, lse=lse, idx=bidx, workspace=bws)
+
     pieces = [("full_select", full)] + [(f"sparse{j}", (lambda j=j: sparse(j)))
                                          for j in range(nsp)]
     pieces += [("decode_select", dsel)] + [(f"decode_sparse{j}", (lambda j=j: dsp(j)))
@@ -263,12 +271,12 @@ def run_ours(args, world, rank, local):
     # gated: they return at once unless a sequence overflowed the sketch
     # candidates); decode sparse 1; overlap 1
     full_launches, dsel_launches = 3, 6
-    launches_per_step = full_launches + nsp + dsel_launches + ndsp + 1
+    launches_per_step = full_launches + nsp + dsel_launches + ndsp + 1 + 3
 
+    extras = [("overlap", overlap), ("full_select_blocks", full_blocks)]
     for _ in range(args.warmup):
-        for _, fn in pieces:
+        for _, fn in pieces + extras:
             fn()
-        overlap()
     # decode step as one CUDA graph (launch-bound inner loop)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
@@ -279,7 +287,8 @@ def run_ours(args, world, rank, local):
 
     times = {name: [] for name, _ in pieces}
     times["decode_step_graph"] = []
-    times["overlap"] = []
+    for name, _ in extras:
+        times[name] = []
     barrier(world)
     with Clocks(local, not args.no_clocks) as clk:
         barrier(world)
@@ -299,12 +308,13 @@ def run_ours(args, world, rank, local):
             g.replay()
             e1.record(stream)
             evs.append(("decode_step_graph", e0, e1))
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            overlap()
-            e1.record(stream)
-            evs.append(("overlap", e0, e1))
+            for name, fn in extras:
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                evs.append((name, e0, e1))
             torch.cuda.synchronize()
             for name, a, b in evs:
                 times[name].append(a.elapsed_time(b))
@@ -320,6 +330,7 @@ def run_ours(args, world, rank, local):
     t_dsp = sum(ms[f"decode_sparse{j}"] for j in range(ndsp)) / ndsp / 1e3
     t_dstep = ms["decode_step_graph"] / 1e3
     t_ovl = ms["overlap"] / 1e3
+    t_blk = ms["full_select_blocks"] / 1e3
     ms_per_step = sum(ms[n] for n, _ in pieces)
 
     value = world * B * L / t_full
@@ -344,6 +355,8 @@ def run_ours(args, world, rank, local):
         roof("decode_sparse", "hbm", dsp_bytes, t_dsp, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
         roof("selection_overlap", "hbm", ovl_bytes, t_ovl, P["hbm"], "GB/s",
              f"hbm_gbs ({P['src']})"),
+        roof("full_attn_select_blocks", "tensor", flops, t_blk, P["bf16_sust"], "TFLOP/s",
+             f"bf16_tflops_sustained ({P['src']})"),
     ]
     kernels[0]["frac_of_burst_peak"] = round(kernels[0]["achieved"] / P["bf16"], 4)
     kernels[0]["work"] = "3*d*Hq*L*(L+1) flops (pass 1 QK^T+PV, pass 2 QK^T)"
@@ -351,6 +364,7 @@ def run_ours(args, world, rank, local):
     kernels[2]["work"] = "B*T*(2d+8) bytes (e4m3 K,V rows + 2 fp32 scales)"
     kernels[3]["work"] = "B*S*(2d+8) bytes"
     kernels[4]["work"] = "B*L*(2*S*4 + 8) bytes (two idx rows in, count and ratio out)"
+    kernels[5]["work"] = "3*d*Hq*L*(L+1) flops (as full_attn_select; 64-token block selection)"
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
@@ -370,6 +384,7 @@ def run_ours(args, world, rank, local):
             "decode_sparse_us": round(t_dsp * 1e6, 1),
             "selection_overlap_us": round(t_ovl * 1e6, 1),
             "selection_overlap_mean": round(float(ratio.double().mean()), 4),
+            "prefill_block_select_tok_s": round(world * B * L / t_blk, 1),
             "ms": {n: round(x, 4) for n, x in ms.items()},
         },
         "roofline": kernels[0],
@@ -377,8 +392,8 @@ def run_ours(args, world, rank, local):
         "gpu_launches": launches_per_step * args.steps + (dsel_launches + ndsp) * args.steps,
         "gpu_launches_note": f"per step: {full_launches} full-select (1 gated re-run) + {nsp} "
                              f"sparse + {dsel_launches} decode-select (2 of them gated "
-                             f"fallbacks) + {ndsp} decode sparse + 1 overlap kernels, plus the "
-                             "same decode kernels replayed in a graph",
+                             f"fallbacks) + {ndsp} decode sparse + 1 overlap + 3 block-selector "
+                             "kernels, plus the same decode kernels replayed in a graph",
         "wall_s_timed_region": round(wall, 3),
     }
 

@@ -457,3 +457,71 @@ def test_block_selector_matches_oracle(cuda_lib, shape):
                                   W=x.W, k_top=x.k)
     ref = oracle.sparse(x.q_sparse[0], x.k_, x.v, idx_t, rows=rows)
     assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d)[rows], ref) <= TOL_BF16
+
+
+# ------------------------------------------- the bench workloads, sampled
+# Full sizes, the launch configuration bench.py times; the oracle recomputes
+# sampled rows (prefill) or sampled sequences (decode) one by one.
+
+def _prefill_rows_128k(L, n_rand, seed):
+    g = np.random.default_rng(seed)
+    fixed = [0, 1, 127, 128, 129, 1151, 1152, 1153, 65536, L - 2, L - 1]
+    return np.unique(np.concatenate([fixed, g.choice(L, n_rand, replace=False)])).astype(np.int64)
+
+
+def test_bench_prefill_128k_sampled(cuda_lib):
+    x = inputs.make_workload("prefill_128k")
+    B, L, Hq, d = x.q.shape
+    q, k, v = cuda(x.q), cuda(x.k_), cuda(x.v)
+    o, lse, idx = cuda_lib.hs2_full_attn_select(q, k, v, x.W, x.k)
+    qs = cuda(x.q_sparse[0])
+    os_ = cuda_lib.hs2_sparse_attn(qs, k, v, idx, W=x.W, k_top=x.k)
+    _, _, bidx = cuda_lib.hs2_full_attn_select_blocks(q, k, v, x.W, x.k, want_lse=False)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    rows = _prefill_rows_128k(L, 13, seed=5)
+    o_r = o.view(B * L, Hq, d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    lse_r = lse.view(B * L, Hq)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    idx_h = idx.view(B * L, -1).cpu().numpy()
+    del q, v, o, lse
+    ora = oracle.full_select(x.q, x.k_, x.v, x.W, x.k, rows=rows, probe=idx_h[rows])
+    assert max_abs(o_r, ora["o"]) <= TOL_BF16
+    assert max_abs(lse_r, ora["lse"]) <= TOL_LSE
+    check_structure(idx_h[rows], rows % L, x.W, x.k)
+    check_selection(idx_h[rows], ora, rows % L, x.W, x.k)
+    # the sparse layer on the GPU's selection (end to end)
+    ref = oracle.sparse(x.q_sparse[0], x.k_, x.v, torch.from_numpy(idx_h).view(B, L, -1),
+                        rows=rows)
+    os_r = os_.view(B * L, Hq, d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
+    assert max_abs(os_r, ref) <= TOL_BF16
+    # the block-level selector on the same rows
+    bora = oracle.block_select(x.q, x.k_, x.v, x.W, x.k, block=64, rows=rows)
+    _check_block_rows(bidx.view(B * L, -1).cpu().numpy(), bora, rows, L, x.W, x.k, 64)
+
+
+@pytest.mark.parametrize("name,seqs", [("decode_256k_b16", [0, 7, 15]), ("decode_1m_b4", [2])])
+def test_bench_decode_sampled(cuda_lib, name, seqs):
+    x = inputs.make_workload(name)
+    B = x.q.shape[0]
+    o, lse, idx = run_decode(cuda_lib, x)
+    # every planted needle of every sequence is selected
+    for b in range(B):
+        assert set(x.needle_pos[b].tolist()) <= set(idx[b].tolist()), b
+    sel = torch.tensor(seqs)
+    ora = oracle.decode_select(x.q[sel], x.k_cache[sel], x.v_cache[sel], x.lengths[sel], x.W,
+                               x.k, kv=x.kv, k_scale=x.k_scale[sel], v_scale=x.v_scale[sel],
+                               probe=idx[seqs])
+    assert max_abs(o[seqs], ora["o"]) <= TOL_E4M3
+    assert max_abs(lse[seqs], ora["lse"]) <= TOL_LSE
+    t = x.lengths[sel].numpy().astype(np.int64) - 1
+    check_structure(idx[seqs], t, x.W, x.k)
+    check_selection(idx[seqs], ora, t, x.W, x.k)
+    # the decode sparse layer on the GPU's selection
+    ods = cuda_lib.hs2_decode_sparse(cuda(x.q_sparse[0]), cuda(x.k_cache), cuda(x.v_cache),
+                                     cuda(x.lengths), cuda(torch.from_numpy(idx)), kv=x.kv,
+                                     k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale),
+                                     W=x.W, k_top=x.k)
+    refd = oracle.decode_sparse(x.q_sparse[0][sel], x.k_cache[sel], x.v_cache[sel],
+                                torch.from_numpy(idx[seqs]), kv=x.kv, k_scale=x.k_scale[sel],
+                                v_scale=x.v_scale[sel])
+    assert max_abs(ods.float().cpu().numpy()[seqs], refd) <= TOL_E4M3

@@ -168,6 +168,10 @@ def hs2_full_attn_select(q, k, v, W: int, k_top: int, *, scale=None, o=None, lse
     return o, lse, idx
 
 
+def hs2_full_attn_select_blocks_workspace(shape: PrefillShape, block: int = 64) -> int:
+    return load().hs2_full_attn_select_blocks_workspace(ctypes.byref(shape), block)
+
+
 def hs2_full_attn_select_blocks(q, k, v, W: int, k_top: int, *, block: int = 64, scale=None,
                                 o=None, lse=None, idx=None, workspace=None, want_lse: bool = True,
                                 stream=None):
@@ -180,7 +184,7 @@ def hs2_full_attn_select_blocks(q, k, v, W: int, k_top: int, *, block: int = 64,
     if lse is None and want_lse:
         lse = torch.empty(B, L, Hq, dtype=torch.float32, device=dev)
     idx = torch.empty(B, L, W + k_top, dtype=torch.int32, device=dev) if idx is None else idx
-    need = load().hs2_full_attn_select_blocks_workspace(ctypes.byref(shape), block)
+    need = hs2_full_attn_select_blocks_workspace(shape, block)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     st = load().hs2_full_attn_select_blocks(ctypes.byref(shape), block, _ptr(q), _ptr(k), _ptr(v),

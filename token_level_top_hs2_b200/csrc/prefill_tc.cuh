@@ -621,8 +621,19 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             const int key0 = kb * SBN + half * 128;
             const bool streams = valid && key0 <= maxkey;
             if constexpr (!BLK) {
+                // the stream has seen kb*128 of the row's n_row candidates and
+                // buffers every one of them at or above its threshold; a
+                // speculative prune keeps 1.5 times their expected share of
+                // the row's top k, plus 32 (on the planted-topic workloads no
+                // row failed the exact check at this margin; at 1.25x + 16 a
+                // few did).  It runs when the buffer is full, and early, as
+                // soon as it holds twice that share plus 256, so the threshold
+                // rises long before the first 2k candidates are buffered.
+                const long long r_own = 3LL * kk * (kb * 128) / (2LL * max(maxkey + 1, 1)) + 32;
+                const bool full = cnt + 128 > cap;
+                const bool early = speculate && r_own < kk && cnt >= 2 * r_own + 256;
                 // make room for this block's 128 candidates before accumulating
-                unsigned need = __ballot_sync(0xffffffffu, streams && cnt + 128 > cap);
+                unsigned need = __ballot_sync(0xffffffffu, streams && (full || early));
                 while (need) {
                     const int src = __ffs(need) - 1;
                     need &= need - 1;
@@ -630,29 +641,26 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         __shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(my_buf), src));
                     const int scnt = __shfl_sync(0xffffffffu, cnt, src);
                     const uint32_t sbase = __shfl_sync(0xffffffffu, max(thr_bits, base_bits), src);
+                    const bool sfull = __shfl_sync(0xffffffffu, full, src);
                     uint32_t ntb = 0;
                     int ncnt = -1;
                     if (speculate) {
-                        // the stream has seen kb*128 of the row's n_row candidates
-                        // and buffers every one of them at or above its threshold;
-                        // keep 1.5 times their expected share of the row's top k,
-                        // plus 32 (on the planted-topic workloads no row failed
-                        // the exact check at this margin; at 1.25x + 16 a few did)
-                        const int n_row = __shfl_sync(0xffffffffu, maxkey + 1, src);
-                        const long long r = 3LL * kk * (kb * 128) / (2LL * max(n_row, 1)) + 32;
+                        const long long r = __shfl_sync(0xffffffffu, r_own, src);
                         // (the histogram prune keeps every key whose score bits
                         // reach the bin of the r-th best; if that frees no room
-                        // the buffer is left as it was and pruned to k below)
+                        // a full buffer is pruned to k below, an early one is
+                        // left as it was)
                         if (r < kk)
                             ncnt = warp_prune(sbuf, scnt, (int)r, cap - 128, sbase, hist, &ntb);
                     }
-                    if (ncnt < 0) ncnt = warp_prune(sbuf, scnt, kk, cap - 128, sbase, hist, &ntb);
-                    if (ncnt < 0) {  // no histogram boundary frees room: exact cut to k
+                    if (ncnt < 0 && sfull)
+                        ncnt = warp_prune(sbuf, scnt, kk, cap - 128, sbase, hist, &ntb);
+                    if (ncnt < 0 && sfull) {  // no histogram boundary frees room: exact cut to k
                         const uint64_t nthr = warp_cut(sbuf, scnt, kk, hist);
                         ntb = (uint32_t)(nthr >> 32);
                         ncnt = kk;
                     }
-                    if (lane == src) {
+                    if (lane == src && ncnt >= 0) {
                         thr_bits = ntb;
                         cnt = ncnt;
                     }
