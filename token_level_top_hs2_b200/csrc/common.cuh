@@ -34,6 +34,13 @@ enum : unsigned {
 
 HS2_DEV uint32_t lane_id() { return threadIdx.x & 31; }
 
+// Three-input maximum (sm_100): one instruction for two comparisons.
+HS2_DEV float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialisation may start while the kernel before it in the stream still
 // runs: griddep_wait() returns once that kernel has completed and its memory

@@ -218,6 +218,8 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 break;
             }
             fence_after_sync();
+            // raw logits; the scale (> 0) is applied once to the max and folded
+            // into the exponent's FMA below
             float x[BN];
 #pragma unroll
             for (int c = 0; c < BN / 32; c++) {
@@ -225,7 +227,7 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 tmem_ld32(s_col + c * 32, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; i++) x[c * 32 + i] = __uint_as_float(r[i]) * scale2;
+                for (int i = 0; i < 32; i++) x[c * 32 + i] = __uint_as_float(r[i]);
             }
             const bool diag = j == n_kt - 1;
             if (diag) {  // diagonal tile: keys j*128 + i, row t = qb*128 + row
@@ -233,9 +235,10 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 for (int i = 0; i < BN; i++)
                     if (i > row) x[i] = -INFINITY;
             }
-            float mx = x[0];
+            float mr = fmaxf(x[0], x[1]);
 #pragma unroll
-            for (int i = 1; i < BN; i++) mx = fmaxf(mx, x[i]);
+            for (int i = 2; i < BN; i += 2) mr = fmax3(mr, x[i], x[i + 1]);
+            const float mx = mr * scale2;
             if (mx > m + kRescaleLog2) {
                 if (j > 0) {
                     const float alpha = ex2(m - mx);
@@ -266,7 +269,8 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 uint32_t w[16];
 #pragma unroll
                 for (int i = 0; i < 16; i++) {
-                    const float p0 = ex2(x[c * 32 + 2 * i] - m), p1 = ex2(x[c * 32 + 2 * i + 1] - m);
+                    const float p0 = ex2(fmaf(x[c * 32 + 2 * i], scale2, -m));
+                    const float p1 = ex2(fmaf(x[c * 32 + 2 * i + 1], scale2, -m));
                     rs += p0 + p1;
                     w[i] = pack_bf16(p0, p1);
                 }
