@@ -135,22 +135,33 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* from the
+    environment); NCCL on GPUs, gloo for host-only checks."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
     if world > 1:
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
 
+def _dev():
+    return "cuda" if torch.cuda.is_available() else "cpu"
+
+
 def max_over_ranks(vals, world):
-    t = torch.tensor(vals, dtype=torch.float64, device="cuda")
+    """Element-wise maximum of a list of floats over all ranks."""
+    t = torch.tensor(vals, dtype=torch.float64, device=_dev())
     if world > 1:
         import torch.distributed as dist
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -161,7 +172,14 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def whole_job_rate(world, units_per_rank, t_max_s):
+    """Weak scaling: every rank processes units_per_rank in its own timed
+    region; the job's rate is all units over the slowest rank's time."""
+    return world * units_per_rank / t_max_s
 
 
 # ------------------------------------------------------------- workloads
@@ -333,7 +351,7 @@ def run_ours(args, world, rank, local):
     t_blk = ms["full_select_blocks"] / 1e3
     ms_per_step = sum(ms[n] for n, _ in pieces)
 
-    value = world * B * L / t_full
+    value = whole_job_rate(world, B * L, t_full)
     flops = prefill_flops(L, Hq, d) * B
     sbytes = sparse_bytes(L, S, d) * B
     dbytes = decode_bytes(Bd, T, dd)
