@@ -17,6 +17,7 @@ own step on its own inputs, with no data-path collective.
 samples of the same workload on the host cores.
 """
 import argparse
+import ctypes
 import datetime
 import hashlib
 import json
@@ -260,6 +261,18 @@ def run_ours(args, world, rank, local):
         for j in range(ndsp):
             dsp(j)
 
+    # the same step with the selected rows staged once for all sparse layers
+    dstaged = torch.empty(hs2.load().hs2_decode_stage_workspace(
+        ctypes.byref(hs2.decode_shape(Bd, T, Hqd, dd, xd.W, xd.k, xd.kv))),
+        dtype=torch.uint8, device=dev)
+
+    def decode_step_staged():
+        dsel()
+        hs2.hs2_decode_stage(kc, vc, lens, didx, Hq=Hqd, W=xd.W, k_top=xd.k, kv=xd.kv,
+                             k_scale=ks, v_scale=vs, staged=dstaged)
+        for j in range(ndsp):
+            hs2.hs2_decode_sparse_staged(dqs[j], dstaged, T, xd.W, xd.k, kv=xd.kv, o=dos)
+
     # cross-layer overlap (diagnostic): the inherited selection against the one
     # the first sparse layer's own queries give, made once outside the timing
     idx_own = torch.empty_like(idx)
@@ -290,6 +303,7 @@ def run_ours(args, world, rank, local):
     # candidates); decode sparse 1; overlap 1
     full_launches, dsel_launches = 3, 6
     launches_per_step = full_launches + nsp + dsel_launches + ndsp + 1 + 3
+    staged_graph_launches = dsel_launches + 1 + ndsp
 
     extras = [("overlap", overlap), ("full_select_blocks", full_blocks)]
     for _ in range(args.warmup):
@@ -300,11 +314,17 @@ def run_ours(args, world, rank, local):
     with torch.cuda.graph(g):
         decode_step()
     g.replay()
+    decode_step_staged()
+    gs = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gs):
+        decode_step_staged()
+    gs.replay()
     torch.cuda.synchronize()
     assert hs2.hs2_get_last_device_error() == 0
 
     times = {name: [] for name, _ in pieces}
     times["decode_step_graph"] = []
+    times["decode_step_graph_staged"] = []
     for name, _ in extras:
         times[name] = []
     barrier(world)
@@ -326,6 +346,12 @@ def run_ours(args, world, rank, local):
             g.replay()
             e1.record(stream)
             evs.append(("decode_step_graph", e0, e1))
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gs.replay()
+            e1.record(stream)
+            evs.append(("decode_step_graph_staged", e0, e1))
             for name, fn in extras:
                 flush.zero_()
                 e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -398,6 +424,7 @@ def run_ours(args, world, rank, local):
             "prefill_sparse_layer_tok_s": round(world * B * L / t_sparse, 1),
             "decode_us_per_step": round(t_dstep * 1e6, 1),
             "decode_us_per_step_unfused_calls": round((t_dsel + ndsp * t_dsp) * 1e6, 1),
+            "decode_us_per_step_staged_rows": round(ms["decode_step_graph_staged"] * 1e3, 1),
             "decode_select_us": round(t_dsel * 1e6, 1),
             "decode_sparse_us": round(t_dsp * 1e6, 1),
             "selection_overlap_us": round(t_ovl * 1e6, 1),
@@ -407,11 +434,13 @@ def run_ours(args, world, rank, local):
         },
         "roofline": kernels[0],
         "kernels": kernels,
-        "gpu_launches": launches_per_step * args.steps + (dsel_launches + ndsp) * args.steps,
+        "gpu_launches": (launches_per_step + dsel_launches + ndsp + staged_graph_launches)
+                        * args.steps,
         "gpu_launches_note": f"per step: {full_launches} full-select (1 gated re-run) + {nsp} "
                              f"sparse + {dsel_launches} decode-select (2 of them gated "
                              f"fallbacks) + {ndsp} decode sparse + 1 overlap + 3 block-selector "
-                             "kernels, plus the same decode kernels replayed in a graph",
+                             "kernels, plus the decode step replayed as two CUDA graphs "
+                             "(gathered rows; rows staged once)",
         "wall_s_timed_region": round(wall, 3),
     }
 

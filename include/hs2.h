@@ -214,6 +214,30 @@ hs2_status hs2_selection_overlap(const hs2_prefill_shape* shape, const int32_t* 
                                  const int32_t* idx_b, int32_t* inter, float* ratio,
                                  hs2_stream_t stream);
 
+/*
+ * Decode step with the selected rows staged once.  Every sparse layer of a
+ * hybrid block reads the K/V rows its full layer selected (KV Reuse, "How it
+ * works"); hs2_decode_stage copies them, per sequence and in idx order, into
+ * a compact buffer, and hs2_decode_sparse_staged runs a decode sparse layer
+ * on it.  Results are bit-identical to hs2_decode_sparse with the same idx.
+ *   hs2_decode_stage_workspace: bytes of the staged buffer for `shape`
+ *     (B * (W+k) * (2 * d * esz + 12) plus alignment; 4.9 MB at B = 16,
+ *     W + k = 1152, e4m3).
+ *   hs2_decode_stage: caches, scales and lengths as hs2_decode_select;
+ *     idx [B, W+k] as it returns (entries in [0, lengths[b]-1] or -1; others
+ *     are skipped and flagged as HS2_ERR_DEVICE_DATA); staged: out.
+ *   hs2_decode_sparse_staged: q [B, Hq, d] bf16 of one sparse layer, the
+ *     staged buffer, o [B, Hq, d] bf16 out.  Any number of layers may reuse
+ *     one staged buffer.
+ */
+size_t hs2_decode_stage_workspace(const hs2_decode_shape* shape);
+hs2_status hs2_decode_stage(const hs2_decode_shape* shape, const void* k_cache,
+                            const void* v_cache, const float* k_scale, const float* v_scale,
+                            const int32_t* lengths, const int32_t* idx, void* staged,
+                            size_t staged_bytes, hs2_stream_t stream);
+hs2_status hs2_decode_sparse_staged(const hs2_decode_shape* shape, const void* q,
+                                    const void* staged, void* o, hs2_stream_t stream);
+
 /* Size of the fixed device scratch used by hs2_decode_select_noalloc. */
 #define HS2_NOALLOC_SCRATCH_BYTES (96u << 20)
 

@@ -525,3 +525,45 @@ def test_bench_decode_sampled(cuda_lib, name, seqs):
                                 torch.from_numpy(idx[seqs]), kv=x.kv, k_scale=x.k_scale[sel],
                                 v_scale=x.v_scale[sel])
     assert max_abs(ods.float().cpu().numpy()[seqs], refd) <= TOL_E4M3
+
+
+# ------------------------------------------- decode step with staged rows
+@pytest.mark.parametrize("kv,B,T,Hq,d,W,k,lengths", [
+    ("e4m3", 5, 12000, 16, 128, 128, 1024, [12000, 7000, 300, 1, 1152]),
+    ("bf16", 3, 5000, 8, 64, 32, 128, [5000, 160, 77]),
+    ("bf16", 2, 3000, 16, 128, 64, 256, None),
+])
+def test_decode_sparse_staged_equals_gathered(cuda_lib, kv, B, T, Hq, d, W, k, lengths):
+    x = _decode_case(kv, B, T, Hq, d, W, k, lengths, seed=inputs.seed_for(3, 11))
+    _, _, idx = run_decode(cuda_lib, x)
+    idx_t = cuda(torch.from_numpy(idx))
+    args = dict(kv=kv, k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale))
+    o_g = cuda_lib.hs2_decode_sparse(cuda(x.q_sparse[0]), cuda(x.k_cache), cuda(x.v_cache),
+                                     cuda(x.lengths), idx_t, W=W, k_top=k, **args)
+    staged = cuda_lib.hs2_decode_stage(cuda(x.k_cache), cuda(x.v_cache), cuda(x.lengths), idx_t,
+                                       Hq=Hq, W=W, k_top=k, **args)
+    o_s = cuda_lib.hs2_decode_sparse_staged(cuda(x.q_sparse[0]), staged, T, W, k, kv=kv)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    # the same rows in the same order: bit-identical
+    assert torch.equal(o_g, o_s)
+    ref = oracle.decode_sparse(x.q_sparse[0], x.k_cache, x.v_cache, torch.from_numpy(idx), kv=kv,
+                               k_scale=x.k_scale, v_scale=x.v_scale)
+    assert max_abs(o_s.float().cpu().numpy(), ref) <= (TOL_E4M3 if kv == "e4m3" else TOL_BF16)
+
+
+def test_decode_stage_flags_out_of_range_entries(cuda_lib):
+    x = _decode_case("e4m3", 2, 4000, 16, 128, 16, 64, [4000, 900], seed=31)
+    _, _, idx = run_decode(cuda_lib, x)
+    bad = idx.copy()
+    bad[1, 20] = 950          # beyond length 900: skipped (staged as -1), flagged
+    staged = cuda_lib.hs2_decode_stage(cuda(x.k_cache), cuda(x.v_cache), cuda(x.lengths),
+                                       cuda(torch.from_numpy(bad)), Hq=16, W=16, k_top=64,
+                                       k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale))
+    assert cuda_lib.hs2_get_last_device_error() == cuda_lib.HS2_ERR_DEVICE_DATA
+    o_s = cuda_lib.hs2_decode_sparse_staged(cuda(x.q_sparse[0]), staged, 4000, 16, 64)
+    bad[1, 20] = -1
+    ref = oracle.decode_sparse(x.q_sparse[0], x.k_cache, x.v_cache, torch.from_numpy(bad),
+                               kv="e4m3", k_scale=x.k_scale, v_scale=x.v_scale)
+    assert max_abs(o_s.float().cpu().numpy(), ref) <= TOL_E4M3
+    assert cuda_lib.hs2_get_last_device_error() == 0

@@ -39,6 +39,7 @@ EXPORTED = [
     "hs2_decode_select", "hs2_decode_sparse", "hs2_get_last_device_error",
     "hs2_decode_select_noalloc", "hs2_selection_overlap",
     "hs2_full_attn_select_blocks_workspace", "hs2_full_attn_select_blocks",
+    "hs2_decode_stage_workspace", "hs2_decode_stage", "hs2_decode_sparse_staged",
 ]
 
 
@@ -96,6 +97,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_decode_sparse.restype = i32
     L.hs2_decode_select_noalloc.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.hs2_decode_select_noalloc.restype = i32
+    L.hs2_decode_stage_workspace.argtypes = [D]
+    L.hs2_decode_stage_workspace.restype = sz
+    L.hs2_decode_stage.argtypes = [D, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    L.hs2_decode_stage.restype = i32
+    L.hs2_decode_sparse_staged.argtypes = [D, vp, vp, vp, vp]
+    L.hs2_decode_sparse_staged.restype = i32
     L.hs2_selection_overlap.argtypes = [P, vp, vp, vp, vp, vp]
     L.hs2_selection_overlap.restype = i32
     L.hs2_get_last_device_error.argtypes = [vp]
@@ -270,6 +277,35 @@ def hs2_selection_overlap(idx_a, idx_b, W: int, k_top: int, *, inter=None, ratio
                                       _ptr(ratio), _stream(stream))
     _check(st, "hs2_selection_overlap")
     return inter, ratio
+
+
+def hs2_decode_stage(k_cache, v_cache, lengths, idx, *, Hq: int, W: int, k_top: int,
+                     kv="e4m3", k_scale=None, v_scale=None, staged=None, stream=None):
+    """Stage the selected rows once for the decode sparse layers.  Returns the
+    staged buffer (uint8, CUDA)."""
+    B, Tmax, d = k_cache.shape
+    shape = decode_shape(B, Tmax, Hq, d, W, k_top, kv)
+    need = load().hs2_decode_stage_workspace(ctypes.byref(shape))
+    if staged is None:
+        staged = torch.empty(max(need, 16), dtype=torch.uint8, device=k_cache.device)
+    st = load().hs2_decode_stage(ctypes.byref(shape), _ptr(_u8(k_cache)), _ptr(_u8(v_cache)),
+                                 _ptr(k_scale), _ptr(v_scale), _ptr(lengths), _ptr(idx),
+                                 _ptr(staged), staged.numel() * staged.element_size(),
+                                 _stream(stream))
+    _check(st, "hs2_decode_stage")
+    return staged
+
+
+def hs2_decode_sparse_staged(q, staged, Tmax: int, W: int, k_top: int, *, kv="e4m3",
+                             scale=None, o=None, stream=None):
+    """One decode sparse layer over staged rows.  q [B,Hq,d] bf16. Returns o."""
+    B, Hq, d = q.shape
+    shape = decode_shape(B, Tmax, Hq, d, W, k_top, kv, scale)
+    o = torch.empty_like(q) if o is None else o
+    st = load().hs2_decode_sparse_staged(ctypes.byref(shape), _ptr(q), _ptr(staged), _ptr(o),
+                                         _stream(stream))
+    _check(st, "hs2_decode_sparse_staged")
+    return o
 
 
 def hs2_get_last_device_error(stream=None) -> int:

@@ -17,6 +17,7 @@
 #include "decode_sketch.cuh"
 #include "decode_tc.cuh"
 #include "overlap.cuh"
+#include "stage.cuh"
 #include "prefill_kernels.cuh"
 #include "prefill_tc.cuh"
 #include "sparse_kernels.cuh"
@@ -765,6 +766,78 @@ hs2_status hs2_decode_sparse(const hs2_decode_shape* shape, const void* q, const
                                              lengths, idx, o, st, flags);
     return run_decode_sparse<64, false>(shape, q, k_cache, v_cache, nullptr, nullptr, lengths,
                                         idx, o, st, flags);
+}
+
+size_t hs2_decode_stage_workspace(const hs2_decode_shape* shape) {
+    if (check_decode(shape) != HS2_OK) return 0;
+    const int esz = shape->kv == HS2_KV_E4M3 ? 1 : 2;
+    return stg::layout(shape->B, shape->W + shape->k, shape->d * esz).total;
+}
+
+hs2_status hs2_decode_stage(const hs2_decode_shape* shape, const void* k_cache,
+                            const void* v_cache, const float* k_scale, const float* v_scale,
+                            const int32_t* lengths, const int32_t* idx, void* staged,
+                            size_t staged_bytes, hs2_stream_t stream) {
+    hs2_status e = check_decode(shape);
+    if (e != HS2_OK) return e;
+    const bool fp8 = shape->kv == HS2_KV_E4M3;
+    if (!k_cache || !v_cache || !lengths || !idx || !staged) return HS2_ERR_INVALID_ARG;
+    if (fp8 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(staged))
+        return HS2_ERR_INVALID_ARG;
+    if (staged_bytes < hs2_decode_stage_workspace(shape)) return HS2_ERR_WORKSPACE;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int S = shape->W + shape->k;
+    const int row_bytes = shape->d * (fp8 ? 1 : 2);
+    const auto* kc = static_cast<const uint8_t*>(k_cache);
+    const auto* vc = static_cast<const uint8_t*>(v_cache);
+    auto* out = static_cast<uint8_t*>(staged);
+    const float* ks = fp8 ? k_scale : nullptr;
+    const float* vs = fp8 ? v_scale : nullptr;
+    if (row_bytes == 128) {
+        const int per_cta = stg::kWarps * (32 / 8) * 4;
+        dim3 grid((S + per_cta - 1) / per_cta, shape->B);
+        stg::stage_rows_kernel<128><<<grid, stg::kWarps * 32, 0, st>>>(
+            kc, vc, ks, vs, lengths, idx, shape->Tmax, S, out, flags);
+    } else {
+        const int per_cta = stg::kWarps * (32 / 16) * 4;
+        dim3 grid((S + per_cta - 1) / per_cta, shape->B);
+        stg::stage_rows_kernel<256><<<grid, stg::kWarps * 32, 0, st>>>(
+            kc, vc, ks, vs, lengths, idx, shape->Tmax, S, out, flags);
+    }
+    return launch_status();
+}
+
+hs2_status hs2_decode_sparse_staged(const hs2_decode_shape* shape, const void* q,
+                                    const void* staged, void* o, hs2_stream_t stream) {
+    hs2_status e = check_decode(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !staged || !o) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(staged) || !aligned16(o)) return HS2_ERR_INVALID_ARG;
+    const bool fp8 = shape->kv == HS2_KV_E4M3;
+    if (fp8 && shape->d != 128) return HS2_ERR_UNSUPPORTED;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int S = shape->W + shape->k;
+    const stg::Layout l = stg::layout(shape->B, S, shape->d * (fp8 ? 1 : 2));
+    const auto* base = static_cast<const uint8_t*>(staged);
+    // the staged rows are a cache of S rows per sequence, the map its index row
+    hs2_decode_shape s2 = *shape;
+    s2.Tmax = S;
+    const void* kc = base + l.k_off;
+    const void* vc = base + l.v_off;
+    const float* ks = reinterpret_cast<const float*>(base + l.sk_off);
+    const float* vs = reinterpret_cast<const float*>(base + l.sv_off);
+    const auto* map = reinterpret_cast<const int32_t*>(base + l.map_off);
+    const auto* len = reinterpret_cast<const int32_t*>(base + l.len_off);
+    if (fp8) return run_decode_sparse<128, true>(&s2, q, kc, vc, ks, vs, len, map, o, st, flags);
+    if (shape->d == 128)
+        return run_decode_sparse<128, false>(&s2, q, kc, vc, nullptr, nullptr, len, map, o, st,
+                                             flags);
+    return run_decode_sparse<64, false>(&s2, q, kc, vc, nullptr, nullptr, len, map, o, st, flags);
 }
 
 hs2_status hs2_selection_overlap(const hs2_prefill_shape* shape, const int32_t* idx_a,
