@@ -32,6 +32,7 @@
 #pragma once
 
 #include "decode_tc.cuh"
+#include "gather_attn.cuh"
 
 namespace hs2 {
 namespace dsk {
@@ -125,7 +126,6 @@ sketch_score_kernel(const uint8_t* __restrict__ sketch, const float* __restrict_
 }
 
 struct GatherShared {
-    float q[16][128];     // f16-rounded query, as the MMA operand saw it
     int cand[kCandCap];   // this CTA's candidate positions
     int hist[260];
     int bin, above;
@@ -161,28 +161,6 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
     const bool ranked = k > 0 && n_cand > k;
     const bool work = ranked && s_end > s_begin;
     griddep_launch();
-    if (work) {
-        // f16-rounded query, 8 elements per thread
-        const __nv_bfloat16* qb = q + (size_t)b * Hq * 128;
-        for (int e = 8 * threadIdx.x; e < 16 * 128; e += 8 * kGatherThreads) {
-            const int h = e >> 7;
-            float4 lo = make_float4(0.f, 0.f, 0.f, 0.f), hi = lo;
-            if (h < Hq) {
-                const uint4 w = *reinterpret_cast<const uint4*>(qb + e);
-                const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
-                float f[8];
-#pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    f[2 * i] = __half2float(__float2half_rn(bf16_lo(wd[i])));
-                    f[2 * i + 1] = __half2float(__float2half_rn(bf16_hi(wd[i])));
-                }
-                lo = make_float4(f[0], f[1], f[2], f[3]);
-                hi = make_float4(f[4], f[5], f[6], f[7]);
-            }
-            *reinterpret_cast<float4*>(&sh.q[h][e & 127]) = lo;
-            *reinterpret_cast<float4*>(&sh.q[h][(e & 127) + 4]) = hi;
-        }
-    }
     // L, its histogram and lse2 come from the kernels before
     griddep_wait();
     if (work) {
@@ -242,63 +220,56 @@ sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigne
         if (nc > kCandCap) {
             if (threadIdx.x == 0) atomicOr(ovf + b, 1u);
         } else {
-            // a thread pair per candidate: lane & 1 takes dims 64 (lane & 1) .. + 63
-            const int half = lane & 1;
-            const int hh = (lane >> 1) & 15;  // the head this lane exponentiates
-            const float l2h = hh < Hq ? __ldcg(lse2_ws + b * 16 + hh) : INFINITY;
+            // a warp per 16 candidates: their K rows go straight into the
+            // fragments of a 16-head x 16-key tensor-core tile (the sparse
+            // layers' warp routine), then sum_h 2^(logit_h - lse2_h) per key
+            const int g = lane >> 2, c = lane & 3;
+            const float l2a = g < Hq ? __ldcg(lse2_ws + b * 16 + g) : INFINITY;
+            const float l2b = g + 8 < Hq ? __ldcg(lse2_ws + b * 16 + g + 8) : INFINITY;
             const uint8_t* kb = kc + (size_t)b * Tmax * 128;
             const float* ksb = ksc + (size_t)b * Tmax;
-            for (int i0 = warp * 16; i0 < nc; i0 += kGatherThreads / 2) {
-                const int i = i0 + (lane >> 1);
-                const bool has = i < nc;
-                const int s = has ? sh.cand[i] : 0;
-                uint4 kw[4];
-                const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)s * 128) + 4 * half;
+            WarpAttn<128, true> wa;
+            wa.load_q(q + (size_t)b * Hq * 128, Hq);  // the range is checked by pass 1
+            constexpr int NW = kGatherThreads / 32;
+            for (int i0 = warp * 16; i0 < nc; i0 += NW * 16) {
+                const int my = (lane < 16 && i0 + lane < nc) ? sh.cand[i0 + lane] : -1;
+                int key_k[2], key_v[4];
+                distribute_keys(my, key_k, key_v);
+                TileRegs<128, true> tr;
+                wa.load_tile(tr, kb, kb, ksb, ksb, key_k, key_v);
+                float sx[2][4];
+                wa.qk(tr, sx);
+                wa.scale_mask(tr, sx, qk2 * 256.f);  // e4m3 rows enter as f16 x 2^-8
+                // this lane: heads g, g+8 of keys 2c, 2c+1 (tile 0), 8+2c, 9+2c (tile 1)
+                float sc[4];
 #pragma unroll
-                for (int c = 0; c < 4; c++) kw[c] = has ? __ldg(kr + c) : make_uint4(0u, 0u, 0u, 0u);
-                const float sk = has ? __ldg(ksb + s) : 0.f;
-                float d[16];
+                for (int j = 0; j < 2; j++)
 #pragma unroll
-                for (int h = 0; h < 16; h++) d[h] = 0.f;
+                    for (int e = 0; e < 2; e++)
+                        sc[2 * j + e] = ex2(sx[j][e] - l2a) + ex2(sx[j][2 + e] - l2b);
 #pragma unroll
-                for (int c = 0; c < 4; c++) {
-                    const uint32_t wd[4] = {kw[c].x, kw[c].y, kw[c].z, kw[c].w};
+                for (int u = 0; u < 4; u++)
 #pragma unroll
-                    for (int m = 0; m < 4; m++) {
-                        const float2 k01 = f16x2_to_float2(e4m3x2_lo_to_f16x2(wd[m]));
-                        const float2 k23 = f16x2_to_float2(e4m3x2_lo_to_f16x2(wd[m] >> 16));
-                        const int dim = 64 * half + 16 * c + 4 * m;
-#pragma unroll
-                        for (int h = 0; h < 16; h++) {
-                            const float4 qv = *reinterpret_cast<const float4*>(&sh.q[h][dim]);
-                            d[h] = fmaf(qv.x, k01.x, d[h]);
-                            d[h] = fmaf(qv.y, k01.y, d[h]);
-                            d[h] = fmaf(qv.z, k23.x, d[h]);
-                            d[h] = fmaf(qv.w, k23.y, d[h]);
-                        }
-                    }
-                }
-                // whole dots on both lanes of the pair
-#pragma unroll
-                for (int h = 0; h < 16; h++) d[h] += __shfl_xor_sync(0xffffffffu, d[h], 1);
-                const float ks = sk * qk2;
-                float sc = 0.f;
-#pragma unroll
-                for (int h = 0; h < 16; h++) {
-                    const float l2 = __shfl_sync(0xffffffffu, l2h, 2 * h);
-                    sc += ex2(fmaf(d[h], ks, -l2));
-                }
-                // one boundary-buffer reservation per warp (even lanes write)
-                const unsigned m = __ballot_sync(0xffffffffu, has && half == 0);
+                    for (int o = 4; o < 32; o <<= 1)
+                        sc[u] += __shfl_xor_sync(0xffffffffu, sc[u], o);
+                // lanes 0..3 hold the sums of the tile's 16 keys; one
+                // boundary-buffer reservation per tile
+                const int n_tile = min(16, nc - i0);
                 unsigned basep = 0;
-                if (lane == 0) basep = atomicAdd(bnd_cnt + b, (unsigned)__popc(m));
+                if (lane == 0) basep = atomicAdd(bnd_cnt + b, (unsigned)n_tile);
                 basep = __shfl_sync(0xffffffffu, basep, 0);
-                if (has && half == 0) {
-                    const unsigned p = basep + (unsigned)__popc(m & ((1u << lane) - 1u));
-                    if (p < (unsigned)dec::BCAP)
-                        bnd[(size_t)b * dec::BCAP + p] = make_key(sc, (uint32_t)s);
-                    else
-                        atomicOr(ovf + b, 1u);
+                if (lane < 4) {
+#pragma unroll
+                    for (int u = 0; u < 4; u++) {
+                        const int col = (u < 2) ? 2 * c + u : 8 + 2 * c + (u - 2);
+                        if (col >= n_tile) continue;
+                        const int pos = sh.cand[i0 + col];
+                        const unsigned p = basep + (unsigned)col;
+                        if (p < (unsigned)dec::BCAP)
+                            bnd[(size_t)b * dec::BCAP + p] = make_key(sc[u], (uint32_t)pos);
+                        else
+                            atomicOr(ovf + b, 1u);
+                    }
                 }
             }
         }
