@@ -381,6 +381,7 @@ gather_kernel(const float* __restrict__ scores, int score_ld, const unsigned* __
     __shared__ GatherShared sh;
     const int b = blockIdx.y, chunk = blockIdx.x;
     // the scores, their histogram and the gate come from the kernels before
+    griddep_launch();
     griddep_wait();
     if (gate != nullptr && __ldcg(gate + b) == 0u) return;
     const int T = __ldg(lengths + b);

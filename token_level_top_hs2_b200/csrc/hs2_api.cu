@@ -598,13 +598,17 @@ hs2_status run_decode_sparse(const hs2_decode_shape* s, const void* q, const voi
     cfg.blockDim = dim3(WARPS * 32);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CLUSTER;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // the launch may overlap the previous kernel's tail (the kernel waits
+    // for it before reading anything)
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, static_cast<const __nv_bfloat16*>(q),
                                        static_cast<const uint8_t*>(kc),
@@ -799,13 +803,15 @@ hs2_status hs2_decode_stage(const hs2_decode_shape* shape, const void* k_cache,
     if (row_bytes == 128) {
         const int per_cta = stg::kWarps * (32 / 8) * 4;
         dim3 grid((S + per_cta - 1) / per_cta, shape->B);
-        stg::stage_rows_kernel<128><<<grid, stg::kWarps * 32, 0, st>>>(
-            kc, vc, ks, vs, lengths, idx, shape->Tmax, S, out, flags);
+        if (launch_pdl(stg::stage_rows_kernel<128>, grid, dim3(stg::kWarps * 32), 0, st, kc, vc,
+                       ks, vs, lengths, idx, shape->Tmax, S, out, flags) != cudaSuccess)
+            return HS2_ERR_CUDA;
     } else {
         const int per_cta = stg::kWarps * (32 / 16) * 4;
         dim3 grid((S + per_cta - 1) / per_cta, shape->B);
-        stg::stage_rows_kernel<256><<<grid, stg::kWarps * 32, 0, st>>>(
-            kc, vc, ks, vs, lengths, idx, shape->Tmax, S, out, flags);
+        if (launch_pdl(stg::stage_rows_kernel<256>, grid, dim3(stg::kWarps * 32), 0, st, kc, vc,
+                       ks, vs, lengths, idx, shape->Tmax, S, out, flags) != cudaSuccess)
+            return HS2_ERR_CUDA;
     }
     return launch_status();
 }

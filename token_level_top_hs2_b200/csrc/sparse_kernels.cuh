@@ -78,6 +78,10 @@ decode_sparse_kernel(const __nv_bfloat16* __restrict__ q, const uint8_t* __restr
     float* wpart = smem_f;                   // WARPS partials
     float* cpart = smem_f + WARPS * PART;    // this CTA's merged partial
 
+    // launched with programmatic serialisation: the launch overlaps the
+    // previous kernel's tail; every input is read after it completed
+    griddep_launch();
+    griddep_wait();
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int b = blockIdx.x / CLUSTER;

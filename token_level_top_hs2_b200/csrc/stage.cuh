@@ -51,6 +51,8 @@ stage_rows_kernel(const uint8_t* __restrict__ kc, const uint8_t* __restrict__ vc
     constexpr int CH = ROW_BYTES / 16;   // 16-byte chunks per row
     constexpr int RPI = 32 / CH;         // rows per warp instruction
     static_assert(ROW_BYTES % 16 == 0 && 32 % CH == 0, "row size");
+    griddep_launch();
+    griddep_wait();  // the selection comes from the kernel before
     const int b = blockIdx.y;
     const int B = gridDim.y;
     const Layout l = layout(B, S, ROW_BYTES);
