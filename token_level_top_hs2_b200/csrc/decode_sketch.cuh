@@ -22,7 +22,8 @@
 // sketch_gather_kernel  the bin holding the k-th largest L gives E, a lower
 //                       bound of the k-th largest score.  A token can be in
 //                       the top k only if 9/8 L + eps >= E; exactly those are
-//                       rescored from their K rows (a thread pair per token); the
+//                       rescored from their K rows (a warp per 16 tokens, one
+//                       16-head x 16-key tensor-core tile); the
 //                       last CTA of the sequence bins their exact scores, takes
 //                       every key above the bin of the k-th and ranks the
 //                       keys inside that bin (ties to the lower position).
