@@ -114,6 +114,23 @@ hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, c
                                 void* workspace, size_t workspace_bytes, hs2_stream_t stream);
 
 /*
+ * The two halves of hs2_full_attn_select, for callers that use the full
+ * layer's output before its selection is done (O and lse are final when
+ * hs2_full_attn returns on the stream; the selection then runs from q, k and
+ * lse): e.g. the next layer, or the copy of O to the host, overlaps the
+ * selection on another stream.  Results equal hs2_full_attn_select's.
+ *   hs2_full_attn: q, k, v, o as hs2_full_attn_select; lse [B, L, Hq] fp32 out
+ *     (required here).
+ *   hs2_select: q, k and the lse hs2_full_attn wrote; idx out; workspace of at
+ *     least hs2_full_attn_select_workspace() bytes.
+ */
+hs2_status hs2_full_attn(const hs2_prefill_shape* shape, const void* q, const void* k,
+                         const void* v, void* o, float* lse, hs2_stream_t stream);
+hs2_status hs2_select(const hs2_prefill_shape* shape, const void* q, const void* k,
+                      const float* lse, int32_t* idx, void* workspace, size_t workspace_bytes,
+                      hs2_stream_t stream);
+
+/*
  * Block-level selector variant: the full layer of HySparse, the predecessor
  * the HySparse2 summary compares against ("Limits": 64-token blocks, 1,024
  * global tokens, a separate 128-token local window).  Same exact attention

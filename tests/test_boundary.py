@@ -131,6 +131,19 @@ def test_decode_rejects_bad_arguments(lib):
              None) == hs2.HS2_ERR_INVALID_ARG
 
 
+def test_split_prefill_calls_reject_bad_arguments(lib):
+    s = hs2.prefill_shape(1, 64, 16, 128, 8, 8)
+    # hs2_full_attn needs lse (the selection reads it)
+    assert lib.hs2_full_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, None,
+                             None) == hs2.HS2_ERR_INVALID_ARG
+    need = hs2.hs2_full_attn_select_workspace(s)
+    f = lib.hs2_select
+    assert f(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == hs2.HS2_ERR_WORKSPACE
+    assert f(ctypes.byref(s), FAKE, FAKE, None, FAKE, FAKE, need, None) == hs2.HS2_ERR_INVALID_ARG
+    bad = hs2.prefill_shape(1, 64, 12, 128, 8, 8)  # 12 query heads: unsupported
+    assert f(ctypes.byref(bad), FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == hs2.HS2_ERR_UNSUPPORTED
+
+
 def test_overlap_rejects_bad_arguments(lib):
     s = hs2.prefill_shape(1, 64, 16, 128, 8, 8)
     f = lib.hs2_selection_overlap

@@ -567,3 +567,16 @@ def test_decode_stage_flags_out_of_range_entries(cuda_lib):
                                kv="e4m3", k_scale=x.k_scale, v_scale=x.v_scale)
     assert max_abs(o_s.float().cpu().numpy(), ref) <= TOL_E4M3
     assert cuda_lib.hs2_get_last_device_error() == 0
+
+
+def test_split_full_attn_and_select_equal_the_combined_call(cuda_lib):
+    x = inputs.make_prefill(2, 777, 16, 128, 128, 256, n_topics=8, seg=256,
+                            seed=inputs.seed_for(0, 5))
+    q, k, v = cuda(x.q), cuda(x.k_), cuda(x.v)
+    o, lse, idx = cuda_lib.hs2_full_attn_select(q, k, v, x.W, x.k)
+    o2, lse2 = cuda_lib.hs2_full_attn(q, k, v)
+    idx2 = cuda_lib.hs2_select(q, k, lse2, x.W, x.k)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    assert torch.equal(torch.sort(idx, dim=-1).values, torch.sort(idx2, dim=-1).values)

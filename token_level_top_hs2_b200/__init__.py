@@ -40,6 +40,7 @@ EXPORTED = [
     "hs2_decode_select_noalloc", "hs2_selection_overlap",
     "hs2_full_attn_select_blocks_workspace", "hs2_full_attn_select_blocks",
     "hs2_decode_stage_workspace", "hs2_decode_stage", "hs2_decode_sparse_staged",
+    "hs2_full_attn", "hs2_select",
 ]
 
 
@@ -83,6 +84,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_full_attn_select_workspace.restype = sz
     L.hs2_full_attn_select.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     L.hs2_full_attn_select.restype = i32
+    L.hs2_full_attn.argtypes = [P, vp, vp, vp, vp, vp, vp]
+    L.hs2_full_attn.restype = i32
+    L.hs2_select.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+    L.hs2_select.restype = i32
     L.hs2_full_attn_select_blocks_workspace.argtypes = [P, i32]
     L.hs2_full_attn_select_blocks_workspace.restype = sz
     L.hs2_full_attn_select_blocks.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -173,6 +178,35 @@ def hs2_full_attn_select(q, k, v, W: int, k_top: int, *, scale=None, o=None, lse
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hs2_full_attn_select")
     return o, lse, idx
+
+
+def hs2_full_attn(q, k, v, *, W: int = 1, k_top: int = 0, scale=None, o=None, lse=None,
+                  stream=None):
+    """Exact causal attention only (O and lse).  Returns (o, lse)."""
+    B, L, Hq, d = q.shape
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    o = torch.empty_like(q) if o is None else o
+    lse = torch.empty(B, L, Hq, dtype=torch.float32, device=q.device) if lse is None else lse
+    st = load().hs2_full_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                              _stream(stream))
+    _check(st, "hs2_full_attn")
+    return o, lse
+
+
+def hs2_select(q, k, lse, W: int, k_top: int, *, scale=None, idx=None, workspace=None,
+               stream=None):
+    """The selection from q, k and the lse of hs2_full_attn.  Returns idx."""
+    B, L, Hq, d = q.shape
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    idx = torch.empty(B, L, W + k_top, dtype=torch.int32, device=q.device) if idx is None else idx
+    need = hs2_full_attn_select_workspace(shape)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    st = load().hs2_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(lse), _ptr(idx),
+                           _ptr(workspace), workspace.numel() * workspace.element_size(),
+                           _stream(stream))
+    _check(st, "hs2_select")
+    return idx
 
 
 def hs2_full_attn_select_blocks_workspace(shape: PrefillShape, block: int = 64) -> int:

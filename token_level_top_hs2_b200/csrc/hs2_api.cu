@@ -246,12 +246,14 @@ BlockWs block_ws(const hs2_prefill_shape* s) {
 template <int D>
 hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void* k,
                            const void* v, void* o, float* lse, int32_t* idx, uint8_t* ws,
-                           cudaStream_t st, unsigned* flags, bool blocks = false) {
+                           cudaStream_t st, unsigned* flags, bool blocks = false,
+                           int phases = 3) {
+    // phases: 1 = exact attention (O, lse), 2 = the selection from lse
     const PrefillWs w = prefill_ws(s);
     const BlockWs bw = block_ws(s);  // same lse area (offset 0) as the token path
     float* lse_p = lse ? lse : reinterpret_cast<float*>(ws + w.lse_off);
     const float scale2 = s->scale * kLog2e;
-    {
+    if (phases & 1) {
         CUtensorMap mq, mk, mv;
         if (!map_q(&mq, q, s->B, s->L, s->Hq, D, tcfa::BM) ||
             !map_kv(&mk, k, s->B, s->L, D, tcfa::BN) || !map_kv(&mv, v, s->B, s->L, D, tcfa::BN))
@@ -264,7 +266,7 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
                                       s->Hq, scale2, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
-    {
+    if (phases & 2) {
         CUtensorMap mq, mk;
         if (!map_q(&mq, q, s->B, s->L, s->Hq, D, tcfa::BM) ||
             !map_kv(&mk, k, s->B, s->L, D, tcfa::SBN))
@@ -660,6 +662,43 @@ hs2_status hs2_full_attn_select(const hs2_prefill_shape* shape, const void* q, c
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     if (shape->d == 128) return run_full_select<128>(shape, q, k, v, o, lse, idx, ws, st, flags);
     return run_full_select<64>(shape, q, k, v, o, lse, idx, ws, st, flags);
+}
+
+hs2_status hs2_full_attn(const hs2_prefill_shape* shape, const void* q, const void* k,
+                         const void* v, void* o, float* lse, hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !k || !v || !o || !lse) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return HS2_ERR_INVALID_ARG;
+    if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (shape->d == 128)
+        return run_full_select<128>(shape, q, k, v, o, lse, nullptr, nullptr, st, flags, false, 1);
+    return run_full_select<64>(shape, q, k, v, o, lse, nullptr, nullptr, st, flags, false, 1);
+}
+
+hs2_status hs2_select(const hs2_prefill_shape* shape, const void* q, const void* k,
+                      const float* lse, int32_t* idx, void* workspace, size_t workspace_bytes,
+                      hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (!q || !k || !lse || !idx || !workspace) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(lse) || !aligned16(idx) ||
+        !aligned16(workspace))
+        return HS2_ERR_INVALID_ARG;
+    if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
+    if (workspace_bytes < prefill_ws(shape).total) return HS2_ERR_WORKSPACE;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* l = const_cast<float*>(lse);  // read only by the selection
+    if (shape->d == 128)
+        return run_full_select<128>(shape, q, k, nullptr, nullptr, l, idx, ws, st, flags, false, 2);
+    return run_full_select<64>(shape, q, k, nullptr, nullptr, l, idx, ws, st, flags, false, 2);
 }
 
 size_t hs2_full_attn_select_blocks_workspace(const hs2_prefill_shape* shape, int block) {
