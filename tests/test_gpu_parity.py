@@ -580,3 +580,40 @@ def test_split_full_attn_and_select_equal_the_combined_call(cuda_lib):
     assert cuda_lib.hs2_get_last_device_error() == 0
     assert torch.equal(o, o2) and torch.equal(lse, lse2)
     assert torch.equal(torch.sort(idx, dim=-1).values, torch.sort(idx2, dim=-1).values)
+
+
+# ------------------------------------------------ the largest index rows
+# W + k = 2048, the largest selection the library accepts.
+
+def test_full_attn_select_largest_selection(cuda_lib):
+    x = inputs.make_prefill(1, 3000, 8, 128, 128, 1920, n_topics=8, seg=256,
+                            seed=inputs.seed_for(0, 21), n_sparse=1)
+    B, L, Hq, d = x.q.shape
+    rows = sample_rows(B, L, 256, seed=4, seg=256)
+    _, idx, ora, rows, n_swap, overlap = check_full_layer(cuda_lib, x, rows=rows)
+    assert overlap > 0.999
+    idx_t = torch.from_numpy(idx).view(B, L, -1)
+    os_ = cuda_lib.hs2_sparse_attn(cuda(x.q_sparse[0]), cuda(x.k_), cuda(x.v), cuda(idx_t),
+                                  W=x.W, k_top=x.k)
+    ref = oracle.sparse(x.q_sparse[0], x.k_, x.v, idx_t, rows=rows)
+    assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d)[rows], ref) <= TOL_BF16
+
+
+def test_decode_select_largest_selection(cuda_lib):
+    x = _decode_case("e4m3", 3, 30000, 16, 128, 1024, 1024, [30000, 12000, 1500],
+                     seed=inputs.seed_for(3, 21))
+    o, lse, idx = run_decode(cuda_lib, x)
+    ora = oracle.decode_select(x.q, x.k_cache, x.v_cache, x.lengths, x.W, x.k, kv="e4m3",
+                               k_scale=x.k_scale, v_scale=x.v_scale, probe=idx)
+    assert max_abs(o, ora["o"]) <= TOL_E4M3
+    assert max_abs(lse, ora["lse"]) <= TOL_LSE
+    t = x.lengths.numpy().astype(np.int64) - 1
+    check_structure(idx, t, x.W, x.k)
+    check_selection(idx, ora, t, x.W, x.k)
+    ods = cuda_lib.hs2_decode_sparse(cuda(x.q_sparse[0]), cuda(x.k_cache), cuda(x.v_cache),
+                                     cuda(x.lengths), cuda(torch.from_numpy(idx)), kv="e4m3",
+                                     k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale),
+                                     W=x.W, k_top=x.k)
+    refd = oracle.decode_sparse(x.q_sparse[0], x.k_cache, x.v_cache, torch.from_numpy(idx),
+                                kv="e4m3", k_scale=x.k_scale, v_scale=x.v_scale)
+    assert max_abs(ods.float().cpu().numpy(), refd) <= TOL_E4M3
