@@ -479,7 +479,7 @@ def test_bench_prefill_128k_sampled(cuda_lib):
     _, _, bidx = cuda_lib.hs2_full_attn_select_blocks(q, k, v, x.W, x.k, want_lse=False)
     torch.cuda.synchronize()
     assert cuda_lib.hs2_get_last_device_error() == 0
-    rows = _prefill_rows_128k(L, 13, seed=5)
+    rows = _prefill_rows_128k(L, 117, seed=5)
     o_r = o.view(B * L, Hq, d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
     lse_r = lse.view(B * L, Hq)[torch.from_numpy(rows).cuda()].cpu().numpy()
     idx_h = idx.view(B * L, -1).cpu().numpy()
@@ -617,3 +617,20 @@ def test_decode_select_largest_selection(cuda_lib):
     refd = oracle.decode_sparse(x.q_sparse[0], x.k_cache, x.v_cache, torch.from_numpy(idx),
                                 kv="e4m3", k_scale=x.k_scale, v_scale=x.v_scale)
     assert max_abs(ods.float().cpu().numpy(), refd) <= TOL_E4M3
+
+
+def test_bench_prefill_32k_three_sparse_layers(cuda_lib):
+    # the 32k workload: the full layer on 512 sampled rows (first 64, last 64,
+    # 64 at segment boundaries, the rest uniform), structure on every row,
+    # and its three sparse layers end to end on the same rows
+    x = inputs.make_workload("prefill_32k")
+    B, L, Hq, d = x.q.shape
+    rows = sample_rows(B, L, 512, seed=7, seg=256)
+    _, idx, ora, rows, n_swap, overlap = check_full_layer(cuda_lib, x, rows=rows)
+    assert overlap > 0.999
+    idx_t = torch.from_numpy(idx).view(B, L, -1)
+    k, v, idx_d = cuda(x.k_), cuda(x.v), cuda(idx_t)
+    for j, qs in enumerate(x.q_sparse):
+        os_ = cuda_lib.hs2_sparse_attn(cuda(qs), k, v, idx_d, W=x.W, k_top=x.k)
+        ref = oracle.sparse(qs, x.k_, x.v, idx_t, rows=rows)
+        assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d)[rows], ref) <= TOL_BF16, j
