@@ -35,7 +35,7 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_agree_on_max_timings():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     want = [2.0, 5.0, 2.5]
     assert out[0] == want and out[1] == want
