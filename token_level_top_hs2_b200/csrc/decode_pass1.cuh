@@ -87,7 +87,7 @@ HS2_DEV void p1_issue_raw(uint8_t* st, const CUtensorMap* mk, const CUtensorMap*
     tma_load_2d(st + P1Layout::RAW_SV, mvs, tok, b, bar);
 }
 
-// grid (n_chunks, B), 384 threads; the last chunk of a sequence to finish
+// grid (n_chunks, B), kP1Threads threads; the last chunk of a sequence to finish
 // merges every chunk's partial into O and lse.
 __global__ void __launch_bounds__(kP1Threads, 1)
 pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,

@@ -134,10 +134,10 @@ struct GatherShared {
 };
 
 // ----------------------------------------------------------------------------
-// Candidates, exact rescoring and the cut.  grid (n_chunks, B), 256 threads,
-// dynamic shared memory BCAP keys (used by the last CTA of each sequence).
-// A thread rescores one candidate at a time from its K row: the same
-// expression the exact pass evaluates, sum_h 2^(<q_h, k_s> sK qk2 - lse2_h).
+// Candidates, exact rescoring and the cut.  grid (n_chunks, B), kGatherThreads
+// threads, dynamic shared memory BCAP keys (used by the last CTA of each
+// sequence).  A warp rescores 16 candidates at a time from their K rows: the
+// same expression the exact pass evaluates, sum_h 2^(<q_h, k_s> sK qk2 - lse2_h).
 __global__ void __launch_bounds__(kGatherThreads)
 sketch_gather_kernel(const float* __restrict__ lrow, int score_ld, const unsigned* __restrict__ hist_g,
                      const uint8_t* __restrict__ kc, const float* __restrict__ ksc,
