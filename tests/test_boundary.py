@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import token_level_top_hs2_b200 as hs2
 from token_level_top_hs2_b200 import build as hs2_build
@@ -166,3 +167,31 @@ def test_binding_fails_loudly_without_library(tmp_path):
             hs2.load(str(tmp_path / "missing.so"))
     finally:
         hs2._lib = saved
+
+
+def test_binding_refuses_host_strided_mistyped_and_missized_tensors(lib):
+    """The binding hands the library raw pointers; anything the kernels would
+    misread (a host tensor, a strided view, another dtype, a wrong extent) is
+    refused on the host before the call."""
+    B, L, Hq, d, W, k = 1, 64, 16, 128, 8, 8
+    q = torch.zeros(B, L, Hq, d, dtype=torch.bfloat16)
+    kv = torch.zeros(B, L, d, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="q: must be a CUDA tensor"):
+        hs2.hs2_full_attn_select(q, kv, kv, W, k)
+    with pytest.raises(ValueError, match="q: must be contiguous"):
+        hs2.hs2_full_attn_select(q.transpose(1, 2).contiguous().transpose(1, 2), kv, kv, W, k)
+    with pytest.raises(ValueError, match="idx_a: must be a CUDA tensor"):
+        idx = torch.zeros(B, L, W + k, dtype=torch.int32)
+        hs2.hs2_selection_overlap(idx, idx, W, k)
+    with pytest.raises(TypeError, match="idx_a: dtype torch.int64"):
+        idx = torch.zeros(B, L, W + k, dtype=torch.int64)
+        hs2.hs2_selection_overlap(idx, idx, W, k)
+    with pytest.raises(ValueError, match="idx_a: 1088 elements, expected 1024"):
+        idx = torch.zeros(B, L, W + k + 1, dtype=torch.int32)
+        hs2.hs2_selection_overlap(idx, idx, W, k)
+    with pytest.raises(TypeError, match="k_cache: dtype torch.bfloat16"):
+        hs2._ptr(kv, "k_cache", hs2._kv_dtypes("e4m3"))
+    assert hs2._kv_dtypes("bf16") == (torch.bfloat16,)
+    with pytest.raises(TypeError, match="expected a torch.Tensor"):
+        hs2._ptr([0], "k")
+    assert hs2._ptr(None, "lse") is None

@@ -120,8 +120,38 @@ def status_string(status: int) -> str:
     return load().hs2_status_string(status).decode()
 
 
-def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+_BF16 = (torch.bfloat16,)
+_F32 = (torch.float32,)
+_I32 = (torch.int32,)
+
+
+def _ptr(t: Optional[torch.Tensor], name: str = "tensor", dtypes=None, numel=None):
+    """Device pointer of a dense CUDA tensor; None stays None (the library
+    rejects a missing required pointer itself).
+
+    The kernels read each argument as a dense row-major array of the type and
+    extent the C header gives, so a host tensor, a strided view, another dtype
+    or a buffer of the wrong size is refused here instead of being misread or
+    overrun on the device."""
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous (dense, row-major)")
+    if dtypes is not None and t.dtype not in dtypes:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor, got device '{t.device}'")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _kv_dtypes(kv):
+    """Element types of K/V storage: bf16 values, or e4m3 codes (as uint8 or
+    float8_e4m3fn)."""
+    return _BF16 if _kv_code(kv) == HS2_KV_BF16 else (torch.uint8, torch.float8_e4m3fn)
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -173,8 +203,12 @@ def hs2_full_attn_select(q, k, v, W: int, k_top: int, *, scale=None, o=None, lse
     need = hs2_full_attn_select_workspace(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    st = load().hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
-                                     _ptr(lse), _ptr(idx), _ptr(workspace),
+    n, nh = B * L * d, B * L * Hq
+    st = load().hs2_full_attn_select(ctypes.byref(shape), _ptr(q, "q", _BF16),
+                                     _ptr(k, "k", _BF16, n), _ptr(v, "v", _BF16, n),
+                                     _ptr(o, "o", _BF16, nh * d), _ptr(lse, "lse", _F32, nh),
+                                     _ptr(idx, "idx", _I32, B * L * (W + k_top)),
+                                     _ptr(workspace, "workspace"),
                                      workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hs2_full_attn_select")
     return o, lse, idx
@@ -187,8 +221,10 @@ def hs2_full_attn(q, k, v, *, W: int = 1, k_top: int = 0, scale=None, o=None, ls
     shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
     o = torch.empty_like(q) if o is None else o
     lse = torch.empty(B, L, Hq, dtype=torch.float32, device=q.device) if lse is None else lse
-    st = load().hs2_full_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                              _stream(stream))
+    n, nh = B * L * d, B * L * Hq
+    st = load().hs2_full_attn(ctypes.byref(shape), _ptr(q, "q", _BF16), _ptr(k, "k", _BF16, n),
+                              _ptr(v, "v", _BF16, n), _ptr(o, "o", _BF16, nh * d),
+                              _ptr(lse, "lse", _F32, nh), _stream(stream))
     _check(st, "hs2_full_attn")
     return o, lse
 
@@ -202,9 +238,11 @@ def hs2_select(q, k, lse, W: int, k_top: int, *, scale=None, idx=None, workspace
     need = hs2_full_attn_select_workspace(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    st = load().hs2_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(lse), _ptr(idx),
-                           _ptr(workspace), workspace.numel() * workspace.element_size(),
-                           _stream(stream))
+    st = load().hs2_select(ctypes.byref(shape), _ptr(q, "q", _BF16),
+                           _ptr(k, "k", _BF16, B * L * d), _ptr(lse, "lse", _F32, B * L * Hq),
+                           _ptr(idx, "idx", _I32, B * L * (W + k_top)),
+                           _ptr(workspace, "workspace"),
+                           workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hs2_select")
     return idx
 
@@ -228,8 +266,13 @@ def hs2_full_attn_select_blocks(q, k, v, W: int, k_top: int, *, block: int = 64,
     need = hs2_full_attn_select_blocks_workspace(shape, block)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    st = load().hs2_full_attn_select_blocks(ctypes.byref(shape), block, _ptr(q), _ptr(k), _ptr(v),
-                                            _ptr(o), _ptr(lse), _ptr(idx), _ptr(workspace),
+    n, nh = B * L * d, B * L * Hq
+    st = load().hs2_full_attn_select_blocks(ctypes.byref(shape), block, _ptr(q, "q", _BF16),
+                                            _ptr(k, "k", _BF16, n), _ptr(v, "v", _BF16, n),
+                                            _ptr(o, "o", _BF16, nh * d),
+                                            _ptr(lse, "lse", _F32, nh),
+                                            _ptr(idx, "idx", _I32, B * L * (W + k_top)),
+                                            _ptr(workspace, "workspace"),
                                             workspace.numel() * workspace.element_size(),
                                             _stream(stream))
     _check(st, "hs2_full_attn_select_blocks")
@@ -245,9 +288,13 @@ def hs2_sparse_attn(q, k, v, idx, *, kv="bf16", k_scale=None, v_scale=None, W=No
         W, k_top = 1, S - 1
     shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
     o = torch.empty_like(q) if o is None else o
-    st = load().hs2_sparse_attn(ctypes.byref(shape), _ptr(q), _ptr(_u8(k)), _ptr(_u8(v)),
-                                _kv_code(kv), _ptr(k_scale), _ptr(v_scale), _ptr(idx), _ptr(o),
-                                _stream(stream))
+    n, kvd = B * L * d, _kv_dtypes(kv)
+    st = load().hs2_sparse_attn(ctypes.byref(shape), _ptr(q, "q", _BF16),
+                                _ptr(_u8(k), "k", kvd, n), _ptr(_u8(v), "v", kvd, n),
+                                _kv_code(kv), _ptr(k_scale, "k_scale", _F32, B * L),
+                                _ptr(v_scale, "v_scale", _F32, B * L),
+                                _ptr(idx, "idx", _I32, B * L * (W + k_top)),
+                                _ptr(o, "o", _BF16, q.numel()), _stream(stream))
     _check(st, "hs2_sparse_attn")
     return o
 
@@ -271,9 +318,16 @@ def hs2_decode_select(q, k_cache, v_cache, lengths, W: int, k_top: int, *, kv="e
     need = hs2_decode_select_workspace(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
-    st = load().hs2_decode_select(ctypes.byref(shape), _ptr(q), _ptr(_u8(k_cache)),
-                                  _ptr(_u8(v_cache)), _ptr(k_scale), _ptr(v_scale),
-                                  _ptr(lengths), _ptr(o), _ptr(lse), _ptr(idx), _ptr(workspace),
+    n, kvd = B * Tmax * d, _kv_dtypes(kv)
+    st = load().hs2_decode_select(ctypes.byref(shape), _ptr(q, "q", _BF16),
+                                  _ptr(_u8(k_cache), "k_cache", kvd, n),
+                                  _ptr(_u8(v_cache), "v_cache", kvd, n),
+                                  _ptr(k_scale, "k_scale", _F32, B * Tmax),
+                                  _ptr(v_scale, "v_scale", _F32, B * Tmax),
+                                  _ptr(lengths, "lengths", _I32, B),
+                                  _ptr(o, "o", _BF16, q.numel()), _ptr(lse, "lse", _F32, B * Hq),
+                                  _ptr(idx, "idx", _I32, B * (W + k_top)),
+                                  _ptr(workspace, "workspace"),
                                   workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hs2_decode_select")
     return o, lse, idx
@@ -289,9 +343,15 @@ def hs2_decode_sparse(q, k_cache, v_cache, lengths, idx, *, kv="e4m3", k_scale=N
         W, k_top = 1, S - 1
     shape = decode_shape(B, Tmax, Hq, d, W, k_top, kv, scale)
     o = torch.empty_like(q) if o is None else o
-    st = load().hs2_decode_sparse(ctypes.byref(shape), _ptr(q), _ptr(_u8(k_cache)),
-                                  _ptr(_u8(v_cache)), _ptr(k_scale), _ptr(v_scale),
-                                  _ptr(lengths), _ptr(idx), _ptr(o), _stream(stream))
+    n, kvd = B * Tmax * d, _kv_dtypes(kv)
+    st = load().hs2_decode_sparse(ctypes.byref(shape), _ptr(q, "q", _BF16),
+                                  _ptr(_u8(k_cache), "k_cache", kvd, n),
+                                  _ptr(_u8(v_cache), "v_cache", kvd, n),
+                                  _ptr(k_scale, "k_scale", _F32, B * Tmax),
+                                  _ptr(v_scale, "v_scale", _F32, B * Tmax),
+                                  _ptr(lengths, "lengths", _I32, B),
+                                  _ptr(idx, "idx", _I32, B * (W + k_top)),
+                                  _ptr(o, "o", _BF16, q.numel()), _stream(stream))
     _check(st, "hs2_decode_sparse")
     return o
 
@@ -307,8 +367,11 @@ def hs2_selection_overlap(idx_a, idx_b, W: int, k_top: int, *, inter=None, ratio
     dev = idx_a.device
     inter = torch.empty(B, L, dtype=torch.int32, device=dev) if inter is None else inter
     ratio = torch.empty(B, L, dtype=torch.float32, device=dev) if ratio is None else ratio
-    st = load().hs2_selection_overlap(ctypes.byref(shape), _ptr(idx_a), _ptr(idx_b), _ptr(inter),
-                                      _ptr(ratio), _stream(stream))
+    S = W + k_top
+    st = load().hs2_selection_overlap(ctypes.byref(shape), _ptr(idx_a, "idx_a", _I32, B * L * S),
+                                      _ptr(idx_b, "idx_b", _I32, B * L * S),
+                                      _ptr(inter, "inter", _I32, B * L),
+                                      _ptr(ratio, "ratio", _F32, B * L), _stream(stream))
     _check(st, "hs2_selection_overlap")
     return inter, ratio
 
@@ -322,9 +385,14 @@ def hs2_decode_stage(k_cache, v_cache, lengths, idx, *, Hq: int, W: int, k_top: 
     need = load().hs2_decode_stage_workspace(ctypes.byref(shape))
     if staged is None:
         staged = torch.empty(max(need, 16), dtype=torch.uint8, device=k_cache.device)
-    st = load().hs2_decode_stage(ctypes.byref(shape), _ptr(_u8(k_cache)), _ptr(_u8(v_cache)),
-                                 _ptr(k_scale), _ptr(v_scale), _ptr(lengths), _ptr(idx),
-                                 _ptr(staged), staged.numel() * staged.element_size(),
+    n, kvd = B * Tmax * d, _kv_dtypes(kv)
+    st = load().hs2_decode_stage(ctypes.byref(shape), _ptr(_u8(k_cache), "k_cache", kvd, n),
+                                 _ptr(_u8(v_cache), "v_cache", kvd, n),
+                                 _ptr(k_scale, "k_scale", _F32, B * Tmax),
+                                 _ptr(v_scale, "v_scale", _F32, B * Tmax),
+                                 _ptr(lengths, "lengths", _I32, B),
+                                 _ptr(idx, "idx", _I32, B * (W + k_top)),
+                                 _ptr(staged, "staged"), staged.numel() * staged.element_size(),
                                  _stream(stream))
     _check(st, "hs2_decode_stage")
     return staged
@@ -336,8 +404,9 @@ def hs2_decode_sparse_staged(q, staged, Tmax: int, W: int, k_top: int, *, kv="e4
     B, Hq, d = q.shape
     shape = decode_shape(B, Tmax, Hq, d, W, k_top, kv, scale)
     o = torch.empty_like(q) if o is None else o
-    st = load().hs2_decode_sparse_staged(ctypes.byref(shape), _ptr(q), _ptr(staged), _ptr(o),
-                                         _stream(stream))
+    st = load().hs2_decode_sparse_staged(ctypes.byref(shape), _ptr(q, "q", _BF16),
+                                         _ptr(staged, "staged"),
+                                         _ptr(o, "o", _BF16, q.numel()), _stream(stream))
     _check(st, "hs2_decode_sparse_staged")
     return o
 
