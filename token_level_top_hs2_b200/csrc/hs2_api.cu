@@ -18,7 +18,6 @@
 #include "decode_tc.cuh"
 #include "overlap.cuh"
 #include "stage.cuh"
-#include "prefill_kernels.cuh"
 #include "prefill_tc.cuh"
 #include "sparse_kernels.cuh"
 
