@@ -451,7 +451,7 @@ def run_ours(args, world, rank, local):
         if clocks:
             line["clocks"] = clocks
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline_prefill(xp, budget_s=15.0)
+            line["cpu_baseline"] = cpu_baseline_prefill(xp, sample_s=15.0)
         print(json.dumps(line), flush=True)
 
 
@@ -507,7 +507,7 @@ def cores_used():
     return oracle.num_threads()
 
 
-def cpu_baseline_prefill(xp, budget_s=15.0, n_rows=None):
+def cpu_baseline_prefill(xp, sample_s=15.0, n_rows=None):
     """fp64 oracle on a bounded sample of query rows of the prefill full+select
     layer, extrapolated to all L rows by causal cost (sum of t+1)."""
     import oracle
@@ -518,7 +518,7 @@ def cpu_baseline_prefill(xp, budget_s=15.0, n_rows=None):
         t0 = time.perf_counter()
         oracle.full_select(xp.q, xp.k_, xp.v, xp.W, xp.k, rows=probe)
         per_full_row = time.perf_counter() - t0
-        n_rows = int(max(4, min(512, 2 * budget_s / max(per_full_row, 1e-6))))
+        n_rows = int(max(4, min(512, 2 * sample_s / max(per_full_row, 1e-6))))
     rows = np.unique(np.linspace(0, L - 1, n_rows).astype(np.int64))
     t0 = time.perf_counter()
     oracle.full_select(xp.q, xp.k_, xp.v, xp.W, xp.k, rows=rows)
