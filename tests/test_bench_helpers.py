@@ -1,0 +1,85 @@
+"""bench.py's host-side measurement arithmetic (no GPU): the algorithmic work
+counts the roofline fractions divide by, the clock-sample summary, and the
+gate that keeps a DRAM-traffic record to the kernel sources it was taken on.
+
+The expected work counts are the per-unit figures of the hot-path scope
+(HySparse2 summary (onedev.kr/papers/146), "How to use": W = 128, k = 1024, MQA,
+d = 128, up to 1M tokens) worked out by hand, not re-derived from bench.py's
+own formulas."""
+import io
+import json
+import os
+
+import pytest
+
+import bench
+
+
+def test_prefill_flops_at_128k():
+    # 6 * d * Hq flops per causal pair (QK^T and PV in the exact pass, QK^T
+    # again in the selection pass) over L(L+1)/2 pairs
+    L, Hq, d = 131072, 16, 128
+    pairs = L * (L + 1) // 2
+    assert bench.prefill_flops(L, Hq, d) == 6 * d * Hq * pairs
+    assert bench.prefill_flops(L, Hq, d) == pytest.approx(1.056e14, rel=1e-3)
+    assert bench.prefill_flops(1, 4, 64) == 6 * 64 * 4  # one pair
+
+
+def test_sparse_bytes_counts_min_t_plus_1_S_rows():
+    # tiny case by enumeration: L = 5, S = 3 -> rows 1, 2, 3, 3, 3
+    assert bench.sparse_bytes(5, 3, 4) == (1 + 2 + 3 + 3 + 3) * 2 * 4 * 2
+    assert bench.sparse_bytes(2, 3, 4) == (1 + 2) * 2 * 4 * 2  # L < S
+    # 128k, S = 1152, bf16: L*S rows less the S(S-1)/2 the first S-1 queries
+    # cannot name, 512 bytes of K+V each; L*S*512 = 77.3 GB is the bound
+    L, S = 131072, 1152
+    assert bench.sparse_bytes(L, S, 128) == (L * S - S * (S - 1) // 2) * 512
+    assert bench.sparse_bytes(L, S, 128) == pytest.approx(77.3e9, rel=5e-3)
+    assert bench.sparse_bytes(131072, 1152, 128, esz=1) * 2 == bench.sparse_bytes(
+        131072, 1152, 128)
+
+
+def test_decode_bytes_264_per_token():
+    # 128 B of K + 128 B of V (e4m3) + two fp32 scales per cached token
+    assert bench.decode_bytes(1, 1, 128) == 264
+    assert bench.decode_bytes(16, 262144, 128) == pytest.approx(1.107e9, rel=1e-3)
+    assert bench.decode_bytes(4, 1 << 20, 128) == bench.decode_bytes(16, 262144, 128)
+
+
+def test_whole_job_rate_is_all_units_over_slowest_rank():
+    assert bench.whole_job_rate(1, 131072, 0.5) == 262144
+    assert bench.whole_job_rate(4, 100, 2.0) == 200
+
+
+def _clocks_from(text):
+    c = bench.Clocks(0, enabled=False)
+    c.proc = object()  # stands for a sampler that ran
+    c.f = io.StringIO(text)
+    return c.summary()
+
+
+def test_clock_summary_median_max_and_active_reasons():
+    rows = [
+        "1900, 1965, 900.1, 0x4, Not Active, Not Active, Not Active, Active",
+        "1920, 1965, 950.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "1930, 1965, 990.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "[N/A], 1965, 0, 0x0, Not Active, Not Active, Not Active, Not Active",  # skipped
+        "short line",
+    ]
+    s = _clocks_from("\n".join(rows) + "\n")
+    assert s["sm_mhz"] == 1920 and s["sm_max_mhz"] == 1965 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    s = _clocks_from("1500, 1965, 700, 0x8, Active, Not Active, Active, Not Active\n")
+    assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert _clocks_from("") is None
+    assert bench.Clocks(0, enabled=False).summary() is None
+
+
+def test_traffic_record_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
+    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
+    # the committed record matches the committed kernel sources
+    assert rec["csrc_hash"] == bench.csrc_hash()
+    assert bench.traffic_for("decode_select") == rec["kernels"]["decode_select"]
+    assert bench.traffic_for("no_such_kernel") is None
+    # a changed source tree invalidates it
+    monkeypatch.setattr(bench, "csrc_hash", lambda: "0000000000000000")
+    assert bench.traffic_for("decode_select") is None
