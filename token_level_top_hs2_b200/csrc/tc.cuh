@@ -68,9 +68,9 @@ HS2_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsi
 }
 
 // ----------------------------------------------------------------------- TMA
-// Tiled tensor loads (no multicast).  The tensor map lives in kernel
-// parameter space (__grid_constant__).  Coordinates are element indices,
-// innermost first.
+// Tiled tensor loads into this CTA's own shared memory.  The tensor map
+// lives in kernel parameter space (__grid_constant__).  Coordinates are
+// element indices, innermost first.
 HS2_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
