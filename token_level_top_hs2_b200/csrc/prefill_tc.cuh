@@ -11,7 +11,8 @@
 //   warps 2-5     softmax of head 0 (thread = query row = TMEM lane; a warp
 //                 reaches TMEM lanes 32*(warp%4)..+31)
 //   warps 6-9     softmax of head 1
-// 320 threads leave 200 registers per thread for the 128-wide rows.
+// 10 warps get at most 168 registers per thread: the register file is split
+// over the SM's four sub-partitions and two of them hold 3 of the warps.
 // TMEM: S0 | S1 | O0 | O1.  The two heads are issued ping-pong so one head's
 // softmax overlaps the other head's GEMMs.  The running max is raised lazily
 // (only when a tile's max exceeds it by more than 2^8), so O is rescaled in
