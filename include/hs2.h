@@ -178,8 +178,11 @@ size_t hs2_decode_select_workspace(const hs2_decode_shape* shape);
 
 /*
  * Decode full layer with selection: one new query per sequence at position
- * t = lengths[b]-1; exact attention over cache rows 0..t and the same
- * selection rule as the prefill call.  Split over the cache length (split-KV).
+ * t = lengths[b]-1; exact attention over cache rows 0..t, and per query the
+ * recent-token window first, then the highest-scoring tokens outside it
+ * (HySparse2 summary, "What differs": token-level selection from exact
+ * attention scores), on the FP8 KV cache the "How to use" section quotes
+ * from 1k to 1M tokens.  Split over the cache length (split-KV).
  *   q        [B, Hq, d] bf16
  *   k_cache, v_cache [B, Tmax, d]  e4m3 codes (kv == HS2_KV_E4M3) or bf16
  *   k_scale, v_scale [B, Tmax] fp32 (e4m3 only; NULL for bf16)
@@ -197,7 +200,10 @@ hs2_status hs2_decode_select(const hs2_decode_shape* shape, const void* q, const
 
 /*
  * Decode sparse layer: sequence b's query attends to the cache rows idx[b]
- * names (KV Reuse of the decode selection).
+ * names -- the sparse layers of a hybrid block reuse the full layer's KV
+ * cache and its token selection unchanged (HySparse2 summary, "How it works",
+ * KV Reuse; "What differs": the sparse layers attend to the tokens the full
+ * layer selected).
  *   q [B, Hq, d] bf16; caches/scales as hs2_decode_select; idx [B, W+k] int32
  *   with entries in [0, lengths[b]-1] or -1; o [B, Hq, d] bf16 out.
  */
@@ -292,6 +298,18 @@ hs2_status hs2_decode_select_noalloc(const hs2_decode_shape* shape, const void* 
                                      const float* k_scale, const float* v_scale,
                                      const int32_t* lengths, void* o, float* lse, int32_t* idx,
                                      hs2_stream_t stream);
+
+/*
+ * hs2_check_bounded_wait: a check of the library's own error path, with no
+ * counterpart in the pages.  Every pipelined kernel waits on its pipeline
+ * stages with a time limit and, when a wait gives up, records a timeout flag
+ * and leaves instead of hanging.  This call launches one warp whose thread 0
+ * waits, through that same bounded wait, on a barrier nothing ever arrives
+ * at, with a limit of `limit_us` microseconds (1 .. 1,000,000); no copy or
+ * tensor-core operation is in flight.  After it, hs2_get_last_device_error
+ * reports HS2_ERR_TIMEOUT once, and the device stays usable.
+ */
+hs2_status hs2_check_bounded_wait(unsigned limit_us, hs2_stream_t stream);
 
 /*
  * Synchronises `stream`, then reports (and clears) the first error met since

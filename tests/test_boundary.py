@@ -195,3 +195,21 @@ def test_binding_refuses_host_strided_mistyped_and_missized_tensors(lib):
     with pytest.raises(TypeError, match="expected a torch.Tensor"):
         hs2._ptr([0], "k")
     assert hs2._ptr(None, "lse") is None
+
+
+def test_binding_refuses_tensors_off_the_current_device(monkeypatch):
+    """The library launches on the current device; a tensor on another GPU is
+    refused on the host (checked here with the current device faked as 0)."""
+    monkeypatch.setattr(hs2, "_current_device", lambda: 0)
+    hs2._check_device("q", torch.device("cuda", 0))
+    hs2._check_device("q", torch.device("cuda"))
+    with pytest.raises(ValueError, match="q: on cuda:1 but the current device is cuda:0"):
+        hs2._check_device("q", torch.device("cuda", 1))
+    with pytest.raises(ValueError, match="k: must be a CUDA tensor"):
+        hs2._check_device("k", torch.device("cpu"))
+
+
+def test_bounded_wait_check_rejects_bad_limits(lib):
+    # refused before anything is launched (no GPU is touched)
+    assert lib.hs2_check_bounded_wait(0, None) == hs2.HS2_ERR_INVALID_ARG
+    assert lib.hs2_check_bounded_wait(1000001, None) == hs2.HS2_ERR_INVALID_ARG

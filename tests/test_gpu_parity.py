@@ -459,72 +459,121 @@ def test_block_selector_matches_oracle(cuda_lib, shape):
     assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d)[rows], ref) <= TOL_BF16
 
 
-# ------------------------------------------- the bench workloads, sampled
-# Full sizes, the launch configuration bench.py times; the oracle recomputes
-# sampled rows (prefill) or sampled sequences (decode) one by one.
+# ------------------------------------------- the bench workloads
+# Full sizes, in the launch configuration bench.py times.  Prefill: the
+# oracle recomputes 512 sampled rows (first 64, last 64, 64 at segment
+# boundaries, the rest uniform) one by one; the structure is checked on
+# every row.  Decode: every sequence of the batch.  The sparse layers are
+# checked end to end (the oracle on the GPU's selection) and in isolation
+# (the GPU kernel fed the oracle's selection on the sampled rows).
 
-def _prefill_rows_128k(L, n_rand, seed):
-    g = np.random.default_rng(seed)
-    fixed = [0, 1, 127, 128, 129, 1151, 1152, 1153, 65536, L - 2, L - 1]
-    return np.unique(np.concatenate([fixed, g.choice(L, n_rand, replace=False)])).astype(np.int64)
+
+def _splice_rows(idx_gpu, rows, idx_rows):
+    """The GPU's [B*L, S] selection with the sampled rows replaced by
+    another selection of those rows (the oracle's)."""
+    out = idx_gpu.copy()
+    out[rows] = idx_rows
+    return out
 
 
-def test_bench_prefill_128k_sampled(cuda_lib):
-    x = inputs.make_workload("prefill_128k")
+def _check_prefill_workload(hs2, name, block_rows=0):
+    x = inputs.make_workload(name)
     B, L, Hq, d = x.q.shape
     q, k, v = cuda(x.q), cuda(x.k_), cuda(x.v)
-    o, lse, idx = cuda_lib.hs2_full_attn_select(q, k, v, x.W, x.k)
-    qs = cuda(x.q_sparse[0])
-    os_ = cuda_lib.hs2_sparse_attn(qs, k, v, idx, W=x.W, k_top=x.k)
-    _, _, bidx = cuda_lib.hs2_full_attn_select_blocks(q, k, v, x.W, x.k, want_lse=False)
+    o, lse, idx = hs2.hs2_full_attn_select(q, k, v, x.W, x.k)
     torch.cuda.synchronize()
-    assert cuda_lib.hs2_get_last_device_error() == 0
-    rows = _prefill_rows_128k(L, 117, seed=5)
-    o_r = o.view(B * L, Hq, d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
-    lse_r = lse.view(B * L, Hq)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    assert hs2.hs2_get_last_device_error() == 0
+    rows = sample_rows(B, L, 512, seed=5, seg=256)
+    assert rows.size >= 500
+    r_dev = torch.from_numpy(rows).cuda()
+    o_r = o.view(B * L, Hq, d)[r_dev].float().cpu().numpy()
+    lse_r = lse.view(B * L, Hq)[r_dev].cpu().numpy()
     idx_h = idx.view(B * L, -1).cpu().numpy()
-    del q, v, o, lse
+    del o, lse
+    check_structure(idx_h, np.tile(np.arange(L), B), x.W, x.k)
     ora = oracle.full_select(x.q, x.k_, x.v, x.W, x.k, rows=rows, probe=idx_h[rows])
     assert max_abs(o_r, ora["o"]) <= TOL_BF16
     assert max_abs(lse_r, ora["lse"]) <= TOL_LSE
-    check_structure(idx_h[rows], rows % L, x.W, x.k)
-    check_selection(idx_h[rows], ora, rows % L, x.W, x.k)
-    # the sparse layer on the GPU's selection (end to end)
-    ref = oracle.sparse(x.q_sparse[0], x.k_, x.v, torch.from_numpy(idx_h).view(B, L, -1),
-                        rows=rows)
-    os_r = os_.view(B * L, Hq, d)[torch.from_numpy(rows).cuda()].float().cpu().numpy()
-    assert max_abs(os_r, ref) <= TOL_BF16
-    # the block-level selector on the same rows
-    bora = oracle.block_select(x.q, x.k_, x.v, x.W, x.k, block=64, rows=rows)
-    _check_block_rows(bidx.view(B * L, -1).cpu().numpy(), bora, rows, L, x.W, x.k, 64)
+    _, overlap = check_selection(idx_h[rows], ora, rows % L, x.W, x.k)
+    assert overlap > 0.999
+    # every sparse layer end to end, on the GPU's selection
+    idx_t = torch.from_numpy(idx_h).view(B, L, -1)
+    for j, qs in enumerate(x.q_sparse):
+        os_ = hs2.hs2_sparse_attn(cuda(qs), k, v, idx, W=x.W, k_top=x.k)
+        ref = oracle.sparse(qs, x.k_, x.v, idx_t, rows=rows)
+        got = os_.view(B * L, Hq, d)[r_dev].float().cpu().numpy()
+        assert max_abs(got, ref) <= TOL_BF16, f"sparse layer {j}"
+    # every sparse layer in isolation: the oracle's selection on the sampled rows
+    mix = torch.from_numpy(_splice_rows(idx_h, rows, ora["idx"])).view(B, L, -1)
+    mix_d = cuda(mix)
+    for j, qs in enumerate(x.q_sparse):
+        os_ = hs2.hs2_sparse_attn(cuda(qs), k, v, mix_d, W=x.W, k_top=x.k)
+        ref = oracle.sparse(qs, x.k_, x.v, mix, rows=rows)
+        got = os_.view(B * L, Hq, d)[r_dev].float().cpu().numpy()
+        assert max_abs(got, ref) <= TOL_BF16, f"sparse layer {j} on the oracle's selection"
+    torch.cuda.synchronize()
+    assert hs2.hs2_get_last_device_error() == 0
+    if block_rows:
+        # the block-level selector on a subset of the same rows
+        brow = rows[np.linspace(0, rows.size - 1, block_rows).astype(np.int64)]
+        _, _, bidx = hs2.hs2_full_attn_select_blocks(q, k, v, x.W, x.k, want_lse=False)
+        bora = oracle.block_select(x.q, x.k_, x.v, x.W, x.k, block=64, rows=brow)
+        _check_block_rows(bidx.view(B * L, -1).cpu().numpy(), bora, brow, L, x.W, x.k, 64)
 
 
-@pytest.mark.parametrize("name,seqs", [("decode_256k_b16", [0, 7, 15]), ("decode_1m_b4", [2])])
-def test_bench_decode_sampled(cuda_lib, name, seqs):
+@pytest.mark.parametrize("repeat", [0, 1, 2])
+def test_tiny_prefill_three_seeds_every_row(cuda_lib, repeat):
+    # the tiny workload (B=1, L=1024, Hq=4, d=64, W=32, k=128), three seeds:
+    # the full layer and its sparse layer on every row, end to end and on the
+    # oracle's selection
+    x = inputs.make_workload("prefill_tiny_1k", repeat=repeat)
+    B, L, Hq, d = x.q.shape
+    _, idx, ora, rows, n_swap, overlap = check_full_layer(cuda_lib, x)
+    assert overlap > 0.999
+    for sel in (idx, ora["idx"]):
+        idx_t = torch.from_numpy(np.ascontiguousarray(sel)).view(B, L, -1)
+        os_ = cuda_lib.hs2_sparse_attn(cuda(x.q_sparse[0]), cuda(x.k_), cuda(x.v), cuda(idx_t),
+                                       W=x.W, k_top=x.k)
+        ref = oracle.sparse(x.q_sparse[0], x.k_, x.v, idx_t)
+        assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d), ref) <= TOL_BF16
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+
+
+def test_bench_prefill_32k_three_sparse_layers(cuda_lib):
+    _check_prefill_workload(cuda_lib, "prefill_32k")
+
+
+def test_bench_prefill_128k_sampled(cuda_lib):
+    _check_prefill_workload(cuda_lib, "prefill_128k", block_rows=96)
+
+
+@pytest.mark.parametrize("name", ["decode_256k_b16", "decode_1m_b4"])
+def test_bench_decode_every_sequence(cuda_lib, name):
     x = inputs.make_workload(name)
-    B = x.q.shape[0]
     o, lse, idx = run_decode(cuda_lib, x)
     # every planted needle of every sequence is selected
-    for b in range(B):
+    for b in range(x.B):
         assert set(x.needle_pos[b].tolist()) <= set(idx[b].tolist()), b
-    sel = torch.tensor(seqs)
-    ora = oracle.decode_select(x.q[sel], x.k_cache[sel], x.v_cache[sel], x.lengths[sel], x.W,
-                               x.k, kv=x.kv, k_scale=x.k_scale[sel], v_scale=x.v_scale[sel],
-                               probe=idx[seqs])
-    assert max_abs(o[seqs], ora["o"]) <= TOL_E4M3
-    assert max_abs(lse[seqs], ora["lse"]) <= TOL_LSE
-    t = x.lengths[sel].numpy().astype(np.int64) - 1
-    check_structure(idx[seqs], t, x.W, x.k)
-    check_selection(idx[seqs], ora, t, x.W, x.k)
-    # the decode sparse layer on the GPU's selection
-    ods = cuda_lib.hs2_decode_sparse(cuda(x.q_sparse[0]), cuda(x.k_cache), cuda(x.v_cache),
-                                     cuda(x.lengths), cuda(torch.from_numpy(idx)), kv=x.kv,
-                                     k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale),
-                                     W=x.W, k_top=x.k)
-    refd = oracle.decode_sparse(x.q_sparse[0][sel], x.k_cache[sel], x.v_cache[sel],
-                                torch.from_numpy(idx[seqs]), kv=x.kv, k_scale=x.k_scale[sel],
-                                v_scale=x.v_scale[sel])
-    assert max_abs(ods.float().cpu().numpy()[seqs], refd) <= TOL_E4M3
+    ora = oracle.decode_select(x.q, x.k_cache, x.v_cache, x.lengths, x.W, x.k, kv=x.kv,
+                               k_scale=x.k_scale, v_scale=x.v_scale, probe=idx)
+    assert max_abs(o, ora["o"]) <= TOL_E4M3
+    assert max_abs(lse, ora["lse"]) <= TOL_LSE
+    t = x.lengths.numpy().astype(np.int64) - 1
+    check_structure(idx, t, x.W, x.k)
+    check_selection(idx, ora, t, x.W, x.k)
+    args = dict(kv=x.kv, k_scale=cuda(x.k_scale), v_scale=cuda(x.v_scale), W=x.W, k_top=x.k)
+    kc, vc, lens = cuda(x.k_cache), cuda(x.v_cache), cuda(x.lengths)
+    for sel, what in ((idx, "the GPU's"), (ora["idx"], "the oracle's")):
+        sel_t = torch.from_numpy(np.ascontiguousarray(sel))
+        for j, qs in enumerate(x.q_sparse):
+            ods = cuda_lib.hs2_decode_sparse(cuda(qs), kc, vc, lens, cuda(sel_t), **args)
+            refd = oracle.decode_sparse(qs, x.k_cache, x.v_cache, sel_t, kv=x.kv,
+                                        k_scale=x.k_scale, v_scale=x.v_scale)
+            assert max_abs(ods.float().cpu().numpy(), refd) <= TOL_E4M3, \
+                f"decode sparse layer {j} on {what} selection"
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
 
 
 # ------------------------------------------- decode step with staged rows
@@ -619,18 +668,17 @@ def test_decode_select_largest_selection(cuda_lib):
     assert max_abs(ods.float().cpu().numpy(), refd) <= TOL_E4M3
 
 
-def test_bench_prefill_32k_three_sparse_layers(cuda_lib):
-    # the 32k workload: the full layer on 512 sampled rows (first 64, last 64,
-    # 64 at segment boundaries, the rest uniform), structure on every row,
-    # and its three sparse layers end to end on the same rows
-    x = inputs.make_workload("prefill_32k")
-    B, L, Hq, d = x.q.shape
-    rows = sample_rows(B, L, 512, seed=7, seg=256)
-    _, idx, ora, rows, n_swap, overlap = check_full_layer(cuda_lib, x, rows=rows)
-    assert overlap > 0.999
-    idx_t = torch.from_numpy(idx).view(B, L, -1)
-    k, v, idx_d = cuda(x.k_), cuda(x.v), cuda(idx_t)
-    for j, qs in enumerate(x.q_sparse):
-        os_ = cuda_lib.hs2_sparse_attn(cuda(qs), k, v, idx_d, W=x.W, k_top=x.k)
-        ref = oracle.sparse(qs, x.k_, x.v, idx_t, rows=rows)
-        assert max_abs(os_.float().cpu().numpy().reshape(B * L, Hq, d)[rows], ref) <= TOL_BF16, j
+def test_bounded_wait_gives_up_and_reports_timeout(cuda_lib):
+    """The bounded wait every pipelined kernel uses: a wait on a barrier that
+    nothing arrives at gives up after its limit (1 ms here), records the
+    timeout, and leaves the device usable -- the next call works and reports
+    no error."""
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    cuda_lib.hs2_check_bounded_wait(1000)
+    assert cuda_lib.hs2_get_last_device_error() == cuda_lib.HS2_ERR_TIMEOUT
+    assert cuda_lib.hs2_get_last_device_error() == 0  # reported once, then cleared
+    x = inputs.make_prefill(1, 300, 16, 128, 16, 32, seed=41)
+    o, lse, idx = run_full(cuda_lib, x)
+    ora = oracle.full_select(x.q, x.k_, x.v, 16, 32, probe=idx)
+    assert max_abs(o, ora["o"]) <= TOL_BF16
+    check_selection(idx, ora, np.arange(300), 16, 32)

@@ -40,7 +40,7 @@ EXPORTED = [
     "hs2_decode_select_noalloc", "hs2_selection_overlap",
     "hs2_full_attn_select_blocks_workspace", "hs2_full_attn_select_blocks",
     "hs2_decode_stage_workspace", "hs2_decode_stage", "hs2_decode_sparse_staged",
-    "hs2_full_attn", "hs2_select",
+    "hs2_full_attn", "hs2_select", "hs2_check_bounded_wait",
 ]
 
 
@@ -110,6 +110,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_decode_sparse_staged.restype = i32
     L.hs2_selection_overlap.argtypes = [P, vp, vp, vp, vp, vp]
     L.hs2_selection_overlap.restype = i32
+    L.hs2_check_bounded_wait.argtypes = [ctypes.c_uint, vp]
+    L.hs2_check_bounded_wait.restype = i32
     L.hs2_get_last_device_error.argtypes = [vp]
     L.hs2_get_last_device_error.restype = i32
     _lib = L
@@ -130,9 +132,10 @@ def _ptr(t: Optional[torch.Tensor], name: str = "tensor", dtypes=None, numel=Non
     rejects a missing required pointer itself).
 
     The kernels read each argument as a dense row-major array of the type and
-    extent the C header gives, so a host tensor, a strided view, another dtype
-    or a buffer of the wrong size is refused here instead of being misread or
-    overrun on the device."""
+    extent the C header gives, so a host tensor, a tensor on a CUDA device other
+    than the current one, a strided view, another dtype or a buffer of the
+    wrong size is refused here instead of being misread or overrun on the
+    device."""
     if t is None:
         return None
     if not isinstance(t, torch.Tensor):
@@ -143,9 +146,25 @@ def _ptr(t: Optional[torch.Tensor], name: str = "tensor", dtypes=None, numel=Non
         raise TypeError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
     if numel is not None and t.numel() != numel:
         raise ValueError(f"{name}: {t.numel()} elements, expected {numel}")
-    if t.device.type != "cuda":
-        raise ValueError(f"{name}: must be a CUDA tensor, got device '{t.device}'")
+    _check_device(name, t.device)
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _current_device() -> int:
+    return torch.cuda.current_device()
+
+
+def _check_device(name: str, device: torch.device) -> None:
+    """The library launches on the current CUDA device (the one cudaGetDevice
+    names) and builds its tensor maps there, so every tensor of a call must
+    live on that device: a pointer into another GPU's memory would reach this
+    GPU's kernels, which without peer access is an illegal address."""
+    if device.type != "cuda":
+        raise ValueError(f"{name}: must be a CUDA tensor, got device '{device}'")
+    cur = _current_device()
+    if device.index is not None and device.index != cur:
+        raise ValueError(f"{name}: on cuda:{device.index} but the current device is cuda:{cur}; "
+                         "make its device current (torch.cuda.device) or move the tensor")
 
 
 def _kv_dtypes(kv):
@@ -409,6 +428,13 @@ def hs2_decode_sparse_staged(q, staged, Tmax: int, W: int, k_top: int, *, kv="e4
                                          _ptr(o, "o", _BF16, q.numel()), _stream(stream))
     _check(st, "hs2_decode_sparse_staged")
     return o
+
+
+def hs2_check_bounded_wait(limit_us: int = 1000, stream=None) -> None:
+    """Launch the check of the bounded in-kernel wait: one thread waits on a
+    barrier nothing arrives at and gives up after limit_us microseconds; the
+    next hs2_get_last_device_error() then returns HS2_ERR_TIMEOUT."""
+    _check(load().hs2_check_bounded_wait(limit_us, _stream(stream)), "hs2_check_bounded_wait")
 
 
 def hs2_get_last_device_error(stream=None) -> int:

@@ -30,10 +30,14 @@ __device__ unsigned g_device_flags;
 
 constexpr int kMaxDevices = 64;
 unsigned* g_flag_ptr[kMaxDevices];
+// guards the per-device address caches (g_flag_ptr, g_noalloc_ptr): host
+// threads may make their first calls on a device at the same time
+std::mutex g_addr_mutex;
 
 unsigned* device_flags() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_addr_mutex);
     if (!g_flag_ptr[dev]) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_flags) != cudaSuccess) return nullptr;
@@ -126,6 +130,22 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Check of the error path every pipelined kernel shares: one thread waits on
+// an mbarrier that nothing arrives at, through the same bounded wait the
+// pipelines use, with a short limit.  No copy or MMA is in flight, so the
+// wait giving up leaves nothing behind; it records FLAG_TIMEOUT.
+__global__ void bounded_wait_check_kernel(unsigned* __restrict__ flags, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_;
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bar, 1);
+        abort_ = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) tc::mbar_wait(&bar, 0, &abort_, flags, limit_ns);
 }
 
 // Zeroes n16 16-byte words; lets the next kernel of the stream launch at once.
@@ -917,6 +937,15 @@ hs2_status hs2_selection_overlap(const hs2_prefill_shape* shape, const int32_t* 
     return launch_status();
 }
 
+hs2_status hs2_check_bounded_wait(unsigned limit_us, hs2_stream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return HS2_ERR_INVALID_ARG;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    bounded_wait_check_kernel<<<1, 32, 0, st>>>(flags, (uint64_t)limit_us * 1000ull);
+    return launch_status();
+}
+
 hs2_status hs2_get_last_device_error(hs2_stream_t stream) {
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(st) != cudaSuccess) return HS2_ERR_CUDA;
@@ -951,6 +980,7 @@ uint8_t* g_noalloc_ptr[kMaxDevices];
 uint8_t* noalloc_scratch() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_addr_mutex);
     if (!g_noalloc_ptr[dev]) {
         uint8_t* ptr = nullptr;
         if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;

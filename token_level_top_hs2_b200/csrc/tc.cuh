@@ -45,20 +45,22 @@ HS2_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for phase `parity` of `bar`, at most kWaitNs nanoseconds.  On timeout
-// (or when another thread of the CTA already gave up: *abort != 0) it records
-// FLAG_TIMEOUT in *flags, sets *abort and returns false; callers then skip the
-// rest of their work and leave through the normal exit path.
+// Wait for phase `parity` of `bar`, at most limit_ns nanoseconds (2 s unless
+// the caller gives another limit).  On timeout (or when another thread of the
+// CTA already gave up: *abort != 0) it records FLAG_TIMEOUT in *flags, sets
+// *abort and returns false; callers then skip the rest of their work and
+// leave through the normal exit path.
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s
 
-HS2_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* flags) {
+HS2_DEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, unsigned* flags,
+                       uint64_t limit_ns = kWaitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = 1;; i++) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;
                 atomicOr(flags, FLAG_TIMEOUT);
                 return false;
