@@ -38,6 +38,9 @@ sys.path.insert(0, ROOT)
 METRIC = "prefill tokens/s (full+select, sparse layer) at 128k; decode µs/step at 256k"
 PREFILL = "prefill_128k"
 DECODE = "decode_256k_b16"
+# the other workloads, each measured after the timed step
+OTHER_PREFILL = ["prefill_tiny_1k", "prefill_32k"]
+OTHER_DECODE = ["decode_1m_b4"]
 N_SPARSE = 3
 FLUSH_BYTES = 256 << 20
 
@@ -53,6 +56,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-clocks", action="store_true")
+    p.add_argument("--no-configs", action="store_true",
+                   help="skip the other workloads measured after the timed step")
     return p.parse_args()
 
 
@@ -203,171 +208,306 @@ def decode_bytes(B, T, d):
     return float(B) * T * (2 * d + 8)
 
 
+class PrefillWork:
+    """One prefill workload resident on the device: the full-attention select
+    layer and its sparse layers reusing the selection and the bf16 KV."""
+
+    def __init__(self, hs2, name, dev, repeat, n_sparse=N_SPARSE):
+        from token_level_top_hs2_b200 import inputs
+        x = inputs.make_workload(name, repeat=repeat)
+        self.name, self.x = name, x
+        self.B, self.L, self.Hq, self.d = B, L, Hq, d = x.q.shape
+        self.W, self.K = W, K = x.W, x.k
+        self.q, self.k, self.v = x.q.to(dev), x.k_.to(dev), x.v.to(dev)
+        self.qs = [t.to(dev) for t in x.q_sparse[:n_sparse]]
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(B, L, Hq, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(B, L, W + K, dtype=torch.int32, device=dev)
+        self.os_ = torch.empty_like(self.q)
+        self.ws = torch.empty(hs2.hs2_full_attn_select_workspace(
+            hs2.prefill_shape(B, L, Hq, d, W, K)), dtype=torch.uint8, device=dev)
+        self.hs2 = hs2
+
+    def full(self):
+        self.hs2.hs2_full_attn_select(self.q, self.k, self.v, self.W, self.K, o=self.o,
+                                      lse=self.lse, idx=self.idx, workspace=self.ws)
+
+    def sparse(self, j):
+        self.hs2.hs2_sparse_attn(self.qs[j], self.k, self.v, self.idx, W=self.W, k_top=self.K,
+                                 o=self.os_)
+
+    def pieces(self, prefix=""):
+        return [(prefix + "full_select", self.full)] + [
+            (prefix + f"sparse{j}", (lambda j=j: self.sparse(j))) for j in range(len(self.qs))]
+
+    def flops(self):
+        return prefill_flops(self.L, self.Hq, self.d) * self.B
+
+    def sparse_bytes(self):
+        return sparse_bytes(self.L, self.W + self.K, self.d) * self.B
+
+
+class DecodeWork:
+    """One decode workload resident on the device: the decode select and its
+    sparse layers over an e4m3 cache with per-token scales."""
+
+    def __init__(self, hs2, name, dev, repeat, n_sparse=N_SPARSE):
+        from token_level_top_hs2_b200 import inputs
+        x = inputs.make_workload(name, repeat=repeat)
+        self.name, self.x = name, x
+        self.B, self.Hq, self.d = B, Hq, d = x.q.shape
+        self.T, self.W, self.K, self.kv = x.Tmax, x.W, x.k, x.kv
+        self.q = x.q.to(dev)
+        self.qs = [t.to(dev) for t in x.q_sparse[:n_sparse]]
+        self.kc, self.vc = x.k_cache.to(dev), x.v_cache.to(dev)
+        self.ks, self.vs = x.k_scale.to(dev), x.v_scale.to(dev)
+        self.lens = x.lengths.to(dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty(B, Hq, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(B, x.W + x.k, dtype=torch.int32, device=dev)
+        self.os_ = torch.empty_like(self.q)
+        self.ws = torch.empty(hs2.hs2_decode_select_workspace(
+            hs2.decode_shape(B, self.T, Hq, d, x.W, x.k, x.kv)), dtype=torch.uint8, device=dev)
+        self.staged = torch.empty(hs2.load().hs2_decode_stage_workspace(
+            ctypes.byref(hs2.decode_shape(B, self.T, Hq, d, x.W, x.k, x.kv))),
+            dtype=torch.uint8, device=dev)
+        self.hs2 = hs2
+        self.graph = self.graph_staged = None
+
+    def select(self):
+        self.hs2.hs2_decode_select(self.q, self.kc, self.vc, self.lens, self.W, self.K,
+                                   kv=self.kv, k_scale=self.ks, v_scale=self.vs, o=self.o,
+                                   lse=self.lse, idx=self.idx, workspace=self.ws)
+
+    def sparse(self, j):
+        self.hs2.hs2_decode_sparse(self.qs[j], self.kc, self.vc, self.lens, self.idx, kv=self.kv,
+                                   k_scale=self.ks, v_scale=self.vs, W=self.W, k_top=self.K,
+                                   o=self.os_)
+
+    def step(self):
+        self.select()
+        for j in range(len(self.qs)):
+            self.sparse(j)
+
+    def step_staged(self):
+        # the same step with the selected rows staged once for all sparse layers
+        self.select()
+        self.hs2.hs2_decode_stage(self.kc, self.vc, self.lens, self.idx, Hq=self.Hq, W=self.W,
+                                  k_top=self.K, kv=self.kv, k_scale=self.ks, v_scale=self.vs,
+                                  staged=self.staged)
+        for j in range(len(self.qs)):
+            self.hs2.hs2_decode_sparse_staged(self.qs[j], self.staged, self.T, self.W, self.K,
+                                              kv=self.kv, o=self.os_)
+
+    def capture(self):
+        """The decode step as CUDA graphs (launch-bound inner loop)."""
+        self.step()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            self.step()
+        self.graph.replay()
+        self.step_staged()
+        self.graph_staged = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph_staged):
+            self.step_staged()
+        self.graph_staged.replay()
+
+    def pieces(self, prefix=""):
+        return ([(prefix + "decode_select", self.select)] +
+                [(prefix + f"decode_sparse{j}", (lambda j=j: self.sparse(j)))
+                 for j in range(len(self.qs))] +
+                [(prefix + "decode_step_graph", lambda: self.graph.replay()),
+                 (prefix + "decode_step_graph_staged", lambda: self.graph_staged.replay())])
+
+    def select_bytes(self):
+        return decode_bytes(self.B, self.T, self.d)
+
+    def sparse_bytes(self):
+        return float(self.B) * (self.W + self.K) * (2 * self.d + 8)
+
+
+def time_pieces(pieces, steps, flush, stream, times):
+    """Time every piece `steps` times with CUDA events on the launching
+    stream, L2 flushed (a 256 MB write) before each."""
+    for _ in range(steps):
+        evs = []
+        for name, fn in pieces:
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            evs.append((name, e0, e1))
+        torch.cuda.synchronize()
+        for name, a, b in evs:
+            times.setdefault(name, []).append(a.elapsed_time(b))
+
+
+def roof(kernel, bound, work, t, peak, unit, peak_src, traffic=None):
+    """Roofline row: achieved = algorithmic work / time against the measured peak."""
+    ach = work / t / (1e12 if unit == "TFLOP/s" else 1e9)
+    return {"kernel": kernel, "bound": bound, "achieved": round(ach, 2), "peak": peak,
+            "unit": unit, "frac": round(ach / peak, 4), "traffic": traffic,
+            "peak_source": peak_src}
+
+
+def gather_roof(kernel, logical_bytes, t, P):
+    """Roofline row of a gather kernel.  achieved = the DRAM bytes ncu measured
+    for this launch (profiles/traffic.json, while the kernel sources match) over
+    the time, against the HBM peak; the logical gathered bytes (rows served from
+    L2 count every time they are read) are reported beside it."""
+    tr = traffic_for(kernel)
+    logical = logical_bytes / t / 1e9
+    if tr is not None:
+        r = roof(kernel, "hbm", tr, t, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})", traffic=tr)
+        r["achieved_basis"] = "measured DRAM bytes per launch / time"
+    else:
+        r = {"kernel": kernel, "bound": "hbm", "achieved": None, "peak": P["hbm"],
+             "unit": "GB/s", "frac": None, "traffic": None,
+             "peak_source": f"hbm_gbs ({P['src']})",
+             "achieved_basis": "no DRAM counters for the current kernel sources"}
+    r["logical_gbs"] = round(logical, 2)
+    r["logical_frac"] = round(logical / P["hbm"], 4)
+    return r
+
+
 def run_ours(args, world, rank, local):
     import token_level_top_hs2_b200 as hs2
-    from token_level_top_hs2_b200 import inputs
 
     hs2.load()
     dev = torch.device("cuda", local)
     P = peaks()
-    xp = inputs.make_workload(args.prefill, repeat=rank)
-    xd = inputs.make_workload(args.decode, repeat=rank)
-    B, L, Hq, d = xp.q.shape
-    W, K = xp.W, xp.k
+    pf = PrefillWork(hs2, args.prefill, dev, rank)
+    dc = DecodeWork(hs2, args.decode, dev, rank)
+    B, L, Hq, d, W, K = pf.B, pf.L, pf.Hq, pf.d, pf.W, pf.K
     S = W + K
-    # device-resident inputs and outputs
-    q, k, v = xp.q.to(dev), xp.k_.to(dev), xp.v.to(dev)
-    qs = [t.to(dev) for t in xp.q_sparse[:N_SPARSE]]
-    nsp = len(qs)
-    o = torch.empty_like(q)
-    lse = torch.empty(B, L, Hq, dtype=torch.float32, device=dev)
-    idx = torch.empty(B, L, S, dtype=torch.int32, device=dev)
-    os_ = torch.empty_like(q)
-    ws = torch.empty(hs2.hs2_full_attn_select_workspace(hs2.prefill_shape(B, L, Hq, d, W, K)),
-                     dtype=torch.uint8, device=dev)
-    Bd, Hqd, dd = xd.q.shape
-    T = xd.Tmax
-    dq = xd.q.to(dev)
-    dqs = [t.to(dev) for t in xd.q_sparse[:N_SPARSE]]
-    ndsp = len(dqs)
-    kc, vc = xd.k_cache.to(dev), xd.v_cache.to(dev)
-    ks, vs = xd.k_scale.to(dev), xd.v_scale.to(dev)
-    lens = xd.lengths.to(dev)
-    do = torch.empty_like(dq)
-    dlse = torch.empty(Bd, Hqd, dtype=torch.float32, device=dev)
-    didx = torch.empty(Bd, xd.W + xd.k, dtype=torch.int32, device=dev)
-    dos = torch.empty_like(dq)
-    dws = torch.empty(hs2.hs2_decode_select_workspace(
-        hs2.decode_shape(Bd, T, Hqd, dd, xd.W, xd.k, xd.kv)), dtype=torch.uint8, device=dev)
+    nsp, ndsp = len(pf.qs), len(dc.qs)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def full():
-        hs2.hs2_full_attn_select(q, k, v, W, K, o=o, lse=lse, idx=idx, workspace=ws)
-
-    def sparse(j):
-        hs2.hs2_sparse_attn(qs[j], k, v, idx, W=W, k_top=K, o=os_)
-
-    def dsel():
-        hs2.hs2_decode_select(dq, kc, vc, lens, xd.W, xd.k, kv=xd.kv, k_scale=ks, v_scale=vs,
-                              o=do, lse=dlse, idx=didx, workspace=dws)
-
-    def dsp(j):
-        hs2.hs2_decode_sparse(dqs[j], kc, vc, lens, didx, kv=xd.kv, k_scale=ks, v_scale=vs,
-                              W=xd.W, k_top=xd.k, o=dos)
-
-    def decode_step():
-        dsel()
-        for j in range(ndsp):
-            dsp(j)
-
-    # the same step with the selected rows staged once for all sparse layers
-    dstaged = torch.empty(hs2.load().hs2_decode_stage_workspace(
-        ctypes.byref(hs2.decode_shape(Bd, T, Hqd, dd, xd.W, xd.k, xd.kv))),
-        dtype=torch.uint8, device=dev)
-
-    def decode_step_staged():
-        dsel()
-        hs2.hs2_decode_stage(kc, vc, lens, didx, Hq=Hqd, W=xd.W, k_top=xd.k, kv=xd.kv,
-                             k_scale=ks, v_scale=vs, staged=dstaged)
-        for j in range(ndsp):
-            hs2.hs2_decode_sparse_staged(dqs[j], dstaged, T, xd.W, xd.k, kv=xd.kv, o=dos)
-
     # cross-layer overlap (diagnostic): the inherited selection against the one
     # the first sparse layer's own queries give, made once outside the timing
-    idx_own = torch.empty_like(idx)
+    idx_own = torch.empty_like(pf.idx)
     inter = torch.empty(B, L, dtype=torch.int32, device=dev)
     ratio = torch.empty(B, L, dtype=torch.float32, device=dev)
-    hs2.hs2_full_attn_select(qs[0], k, v, W, K, o=os_, lse=lse, idx=idx_own, workspace=ws)
+    hs2.hs2_full_attn_select(pf.qs[0], pf.k, pf.v, W, K, o=pf.os_, lse=pf.lse, idx=idx_own,
+                             workspace=pf.ws)
 
     def overlap():
-        hs2.hs2_selection_overlap(idx, idx_own, W, K, inter=inter, ratio=ratio)
+        hs2.hs2_selection_overlap(pf.idx, idx_own, W, K, inter=inter, ratio=ratio)
 
     # HySparse's block-level selector on the same layer (64-token blocks)
     bws = torch.empty(hs2.hs2_full_attn_select_blocks_workspace(
         hs2.prefill_shape(B, L, Hq, d, W, K), 64), dtype=torch.uint8, device=dev)
-    bidx = torch.empty_like(idx)
+    bidx = torch.empty_like(pf.idx)
 
     def full_blocks():
-        hs2.hs2_full_attn_select_blocks(q, k, v, W, K, o=o, lse=lse, idx=bidx, workspace=bws)
+        hs2.hs2_full_attn_select_blocks(pf.q, pf.k, pf.v, W, K, o=pf.o, lse=pf.lse, idx=bidx,
+                                        workspace=bws)
 
-    pieces = [("full_select", full)] + [(f"sparse{j}", (lambda j=j: sparse(j)))
-                                         for j in range(nsp)]
-    pieces += [("decode_select", dsel)] + [(f"decode_sparse{j}", (lambda j=j: dsp(j)))
-                                          for j in range(ndsp)]
+    # the other workloads, measured after the timed step: the tiny and 32k
+    # prefills and the 1M-token decode (each rank its own inputs)
+    others = []
+    if not args.no_configs:
+        for name in OTHER_PREFILL:
+            if name != args.prefill:
+                others.append(PrefillWork(hs2, name, dev, rank))
+        for name in OTHER_DECODE:
+            if name != args.decode:
+                others.append(DecodeWork(hs2, name, dev, rank))
+
     # kernels per call: full select 3 (pass 1, pass 2 + selection, and pass 2
     # again gated: it returns at once unless a query block failed the check of
     # its speculative thresholds); sparse 1; decode select 6 (workspace zeroing,
     # pass 1, sketch score, sketch gather, and the exact pass 2 and gather,
     # gated: they return at once unless a sequence overflowed the sketch
-    # candidates); decode sparse 1; overlap 1
+    # candidates); decode sparse 1; stage 1; overlap 1; block selector 3
     full_launches, dsel_launches = 3, 6
-    launches_per_step = full_launches + nsp + dsel_launches + ndsp + 1 + 3
-    staged_graph_launches = dsel_launches + 1 + ndsp
 
+    def launches(work):
+        if isinstance(work, PrefillWork):
+            return full_launches + len(work.qs)
+        n = len(work.qs)
+        # the eager calls, then the two graphs (gathered rows; rows staged once)
+        return (dsel_launches + n) * 2 + dsel_launches + 1 + n
+
+    step_pieces = pf.pieces() + dc.pieces()[:1 + ndsp]
+    graph_pieces = dc.pieces()[1 + ndsp:]
     extras = [("overlap", overlap), ("full_select_blocks", full_blocks)]
     for _ in range(args.warmup):
-        for _, fn in pieces + extras:
+        for _, fn in step_pieces + extras:
             fn()
-    # decode step as one CUDA graph (launch-bound inner loop)
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        decode_step()
-    g.replay()
-    decode_step_staged()
-    gs = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gs):
-        decode_step_staged()
-    gs.replay()
+    dc.capture()
     torch.cuda.synchronize()
     assert hs2.hs2_get_last_device_error() == 0
 
-    times = {name: [] for name, _ in pieces}
-    times["decode_step_graph"] = []
-    times["decode_step_graph_staged"] = []
-    for name, _ in extras:
-        times[name] = []
+    times = {}
     barrier(world)
     with Clocks(local, not args.no_clocks) as clk:
         barrier(world)
         t_wall = time.perf_counter()
-        for _ in range(args.steps):
-            evs = []
-            for name, fn in pieces:
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                fn()
-                e1.record(stream)
-                evs.append((name, e0, e1))
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-            evs.append(("decode_step_graph", e0, e1))
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            gs.replay()
-            e1.record(stream)
-            evs.append(("decode_step_graph_staged", e0, e1))
-            for name, fn in extras:
-                flush.zero_()
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                fn()
-                e1.record(stream)
-                evs.append((name, e0, e1))
-            torch.cuda.synchronize()
-            for name, a, b in evs:
-                times[name].append(a.elapsed_time(b))
+        time_pieces(step_pieces + graph_pieces + extras, args.steps, flush, stream, times)
         barrier(world)
         wall = time.perf_counter() - t_wall
     assert hs2.hs2_get_last_device_error() == 0
+    n_launch = (launches(pf) + launches(dc) + 1 + 3) * args.steps
+
+    # the other workloads: warm-up, then the same number of timed repetitions
+    for w in others:
+        if isinstance(w, DecodeWork):
+            for _ in range(args.warmup):
+                w.step()
+            w.capture()
+        else:
+            for _ in range(args.warmup):
+                for _, fn in w.pieces():
+                    fn()
+        torch.cuda.synchronize()
+        time_pieces(w.pieces(w.name + "/"), args.steps, flush, stream, times)
+        n_launch += launches(w) * args.steps
+    assert hs2.hs2_get_last_device_error() == 0
+
     names = list(times)
     avg = max_over_ranks([sum(times[n]) / len(times[n]) for n in names], world)
     ms = dict(zip(names, avg))
+
+    def prefill_summary(w, prefix=""):
+        t_full = ms[prefix + "full_select"] / 1e3
+        t_sp = sum(ms[prefix + f"sparse{j}"] for j in range(len(w.qs))) / len(w.qs) / 1e3
+        r = roof("full_attn_select", "tensor", w.flops(), t_full, P["bf16"], "TFLOP/s",
+                 f"bf16_tflops, burst ({P['src']})")
+        return {"workload": w.name, "B": w.B, "L": w.L, "Hq": w.Hq, "d": w.d, "W": w.W,
+                "k": w.K, "full_select_ms": round(t_full * 1e3, 4),
+                "full_select_tok_s": round(world * w.B * w.L / t_full, 1),
+                "full_select_tflops": r["achieved"], "full_select_frac_of_burst": r["frac"],
+                "full_select_frac_of_sustained": round(r["achieved"] / P["bf16_sust"], 4),
+                "sparse_layer_ms": round(t_sp * 1e3, 4),
+                "sparse_layer_tok_s": round(world * w.B * w.L / t_sp, 1),
+                "sparse_logical_gbs": round(w.sparse_bytes() / t_sp / 1e9, 1),
+                "n_sparse_layers": len(w.qs)}
+
+    def decode_summary(w, prefix=""):
+        t_sel = ms[prefix + "decode_select"] / 1e3
+        t_sp = sum(ms[prefix + f"decode_sparse{j}"] for j in range(len(w.qs))) / len(w.qs) / 1e3
+        t_step = ms[prefix + "decode_step_graph"] / 1e3
+        return {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "d": w.d, "W": w.W,
+                "k": w.K, "kv": w.kv, "us_per_step": round(t_step * 1e6, 1),
+                "us_per_step_unfused_calls": round((t_sel + len(w.qs) * t_sp) * 1e6, 1),
+                "us_per_step_staged_rows": round(ms[prefix + "decode_step_graph_staged"] * 1e3,
+                                                 1),
+                "select_us": round(t_sel * 1e6, 1),
+                "select_gbs": round(w.select_bytes() / t_sel / 1e9, 1),
+                "select_frac_of_hbm": round(w.select_bytes() / t_sel / 1e9 / P["hbm"], 4),
+                "sparse_layer_us": round(t_sp * 1e6, 1),
+                "sparse_gbs": round(w.sparse_bytes() / t_sp / 1e9, 1),
+                "sparse_frac_of_hbm": round(w.sparse_bytes() / t_sp / 1e9 / P["hbm"], 4),
+                "n_sparse_layers": len(w.qs)}
+
+    cfg = {pf.name: prefill_summary(pf), dc.name: decode_summary(dc)}
+    for w in others:
+        cfg[w.name] = (prefill_summary(w, w.name + "/") if isinstance(w, PrefillWork)
+                       else decode_summary(w, w.name + "/"))
+
     t_full = ms["full_select"] / 1e3
     t_sparse = sum(ms[f"sparse{j}"] for j in range(nsp)) / nsp / 1e3
     t_dsel = ms["decode_select"] / 1e3
@@ -375,34 +515,24 @@ def run_ours(args, world, rank, local):
     t_dstep = ms["decode_step_graph"] / 1e3
     t_ovl = ms["overlap"] / 1e3
     t_blk = ms["full_select_blocks"] / 1e3
-    ms_per_step = sum(ms[n] for n, _ in pieces)
+    ms_per_step = sum(ms[n] for n, _ in step_pieces)
 
     value = whole_job_rate(world, B * L, t_full)
-    flops = prefill_flops(L, Hq, d) * B
-    sbytes = sparse_bytes(L, S, d) * B
-    dbytes = decode_bytes(Bd, T, dd)
-    dsp_bytes = float(Bd) * (xd.W + xd.k) * (2 * dd + 8)
     ovl_bytes = float(B) * L * (2 * S * 4 + 8)
-
-    def roof(kernel, bound, work, t, peak, unit, peak_src):
-        ach = work / t / (1e12 if unit == "TFLOP/s" else 1e9)
-        tr = traffic_for(kernel)
-        return {"kernel": kernel, "bound": bound, "achieved": round(ach, 2),
-                "peak": peak, "unit": unit, "frac": round(ach / peak, 4),
-                "traffic": tr, "peak_source": peak_src}
-
+    burst = f"bf16_tflops, burst: the kernel is timed alone ({P['src']})"
     kernels = [
-        roof("full_attn_select", "tensor", flops, t_full, P["bf16_sust"], "TFLOP/s",
-             f"bf16_tflops_sustained ({P['src']})"),
-        roof("sparse_attn", "hbm", sbytes, t_sparse, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
-        roof("decode_select", "hbm", dbytes, t_dsel, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
-        roof("decode_sparse", "hbm", dsp_bytes, t_dsp, P["hbm"], "GB/s", f"hbm_gbs ({P['src']})"),
-        roof("selection_overlap", "hbm", ovl_bytes, t_ovl, P["hbm"], "GB/s",
-             f"hbm_gbs ({P['src']})"),
-        roof("full_attn_select_blocks", "tensor", flops, t_blk, P["bf16_sust"], "TFLOP/s",
-             f"bf16_tflops_sustained ({P['src']})"),
+        roof("full_attn_select", "tensor", pf.flops(), t_full, P["bf16"], "TFLOP/s", burst,
+             traffic_for("full_attn_select")),
+        gather_roof("sparse_attn", pf.sparse_bytes(), t_sparse, P),
+        roof("decode_select", "hbm", dc.select_bytes(), t_dsel, P["hbm"], "GB/s",
+             f"hbm_gbs ({P['src']})", traffic_for("decode_select")),
+        gather_roof("decode_sparse", dc.sparse_bytes(), t_dsp, P),
+        gather_roof("selection_overlap", ovl_bytes, t_ovl, P),
+        roof("full_attn_select_blocks", "tensor", pf.flops(), t_blk, P["bf16"], "TFLOP/s", burst,
+             traffic_for("full_attn_select_blocks")),
     ]
-    kernels[0]["frac_of_burst_peak"] = round(kernels[0]["achieved"] / P["bf16"], 4)
+    for kk in (kernels[0], kernels[5]):
+        kk["frac_of_sustained_peak"] = round(kk["achieved"] / P["bf16_sust"], 4)
     kernels[0]["work"] = "3*d*Hq*L*(L+1) flops (pass 1 QK^T+PV, pass 2 QK^T)"
     kernels[1]["work"] = "sum_t min(t+1,S)*2*d*2 logical gathered bytes"
     kernels[2]["work"] = "B*T*(2d+8) bytes (e4m3 K,V rows + 2 fp32 scales)"
@@ -417,8 +547,8 @@ def run_ours(args, world, rank, local):
         "data": "synthetic (seeded planted-topic prefill, needle decode; no datasets)",
         "config": {"workload": f"{args.prefill} + {args.decode}", "prefill_B": B, "L": L,
                    "Hq": Hq, "d": d, "W": W, "k": K, "n_sparse_layers": nsp,
-                   "decode_B": Bd, "T": T, "kv_decode": xd.kv, "l2": "flushed (256 MB write) "
-                   "before every timed kernel", "parallelism": f"replicas x{world}"},
+                   "decode_B": dc.B, "T": dc.T, "kv_decode": dc.kv, "l2": "flushed (256 MB "
+                   "write) before every timed kernel", "parallelism": f"replicas x{world}"},
         "components": {
             "prefill_full_select_tok_s": round(world * B * L / t_full, 1),
             "prefill_sparse_layer_tok_s": round(world * B * L / t_sparse, 1),
@@ -430,28 +560,28 @@ def run_ours(args, world, rank, local):
             "selection_overlap_us": round(t_ovl * 1e6, 1),
             "selection_overlap_mean": round(float(ratio.double().mean()), 4),
             "prefill_block_select_tok_s": round(world * B * L / t_blk, 1),
+            "configs": cfg,
             "ms": {n: round(x, 4) for n, x in ms.items()},
         },
         "roofline": kernels[0],
         "kernels": kernels,
-        "gpu_launches": (launches_per_step + dsel_launches + ndsp + staged_graph_launches)
-                        * args.steps,
-        "gpu_launches_note": f"per step: {full_launches} full-select (1 gated re-run) + {nsp} "
+        "gpu_launches": n_launch,
+        "gpu_launches_note": f"timed step: {full_launches} full-select (1 gated re-run) + {nsp} "
                              f"sparse + {dsel_launches} decode-select (2 of them gated "
-                             f"fallbacks) + {ndsp} decode sparse + 1 overlap + 3 block-selector "
-                             "kernels, plus the decode step replayed as two CUDA graphs "
-                             "(gathered rows; rows staged once)",
+                             f"fallbacks) + {ndsp} decode sparse, the decode step replayed as "
+                             "two CUDA graphs (gathered rows; rows staged once), 1 overlap + 3 "
+                             "block-selector kernels; then the other workloads' calls",
         "wall_s_timed_region": round(wall, 3),
     }
 
     if not args.no_e2e:
-        line["e2e"] = e2e_prefill(hs2, xp, args, world, dev, W, K, ws, flush)
+        line["e2e"] = e2e_prefill(hs2, pf.x, args, world, dev, W, K, pf.ws, flush)
     if rank == 0:
         clocks = clk.summary()
         if clocks:
             line["clocks"] = clocks
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline_prefill(xp, sample_s=15.0)
+            line["cpu_baseline"] = cpu_baseline(pf.x, dc.x, sample_s=15.0)
         print(json.dumps(line), flush=True)
 
 
@@ -527,8 +657,57 @@ def cpu_baseline_prefill(xp, sample_s=15.0, n_rows=None):
     t_full = dt / frac
     return {"value": round(B * L / (t_full * B), 1), "unit": "tokens/s", "cores": cores_used(),
             "kind": "oracle",
-            "sample": f"{rows.size} evenly spaced query rows of the 128k full+select layer "
-                      f"({dt:.1f} s fp64), extrapolated to all {L} rows by causal cost"}
+            "sample": f"{rows.size} evenly spaced query rows of the {L}-token full+select "
+                      f"layer ({dt:.1f} s fp64), extrapolated to all rows by causal cost"}
+
+
+def cpu_baseline_sparse(xp, n_rows=4096):
+    """fp64 oracle of one sparse layer on a sample of query rows past the first
+    W+k (each of those attends to exactly W+k rows, so the per-row cost is the
+    same for every such row), scaled to all L rows."""
+    import oracle
+    B, L, Hq, d = xp.q.shape
+    S = xp.W + xp.k
+    rows = np.unique(np.linspace(min(S, L - 1), L - 1, n_rows).astype(np.int64))
+    # the selection the layer reuses: the window plus the k positions before it
+    # (what it attends to does not change the cost per row)
+    idx = np.full((B * L, S), -1, dtype=np.int32)
+    for r in rows:
+        t = int(r % L)
+        n = min(t + 1, S)
+        idx[r, :n] = np.arange(t - n + 1, t + 1)
+    t0 = time.perf_counter()
+    oracle.sparse(xp.q_sparse[0], xp.k_, xp.v, idx, rows=rows)
+    dt = time.perf_counter() - t0
+    return {"value": round(B * L / (dt * B * L / rows.size), 1), "unit": "tokens/s",
+            "sample": f"{rows.size} query rows of one sparse layer ({dt:.2f} s fp64), "
+                      f"scaled to all {L} rows"}
+
+
+def cpu_baseline_decode(xd, n_sparse=N_SPARSE):
+    """fp64 oracle of the whole decode step (select over every sequence, then
+    the sparse layers on its selection)."""
+    import oracle
+    t0 = time.perf_counter()
+    ora = oracle.decode_select(xd.q, xd.k_cache, xd.v_cache, xd.lengths, xd.W, xd.k, kv=xd.kv,
+                               k_scale=xd.k_scale, v_scale=xd.v_scale)
+    sel = torch.from_numpy(ora["idx"])
+    for qs in xd.q_sparse[:n_sparse]:
+        oracle.decode_sparse(qs, xd.k_cache, xd.v_cache, sel, kv=xd.kv, k_scale=xd.k_scale,
+                             v_scale=xd.v_scale)
+    dt = time.perf_counter() - t0
+    return {"value": round(dt * 1e6, 1), "unit": "us/step",
+            "sample": f"the whole step: {xd.B} sequences x {xd.Tmax} tokens, select + "
+                      f"{len(xd.q_sparse[:n_sparse])} sparse layers ({dt:.1f} s fp64)"}
+
+
+def cpu_baseline(xp, xd, sample_s=15.0):
+    """The oracle as the CPU baseline: prefill full+select tokens/s (the
+    headline), with the decode step and one sparse layer beside it."""
+    r = cpu_baseline_prefill(xp, sample_s=sample_s)
+    r["components"] = {"decode_us_per_step": cpu_baseline_decode(xd),
+                       "prefill_sparse_layer_tok_s": cpu_baseline_sparse(xp)}
+    return r
 
 
 def run_reference(args):
@@ -537,19 +716,25 @@ def run_reference(args):
     xp = inputs.make_workload(args.prefill)
     B, L, Hq, d = xp.q.shape
     rows_per_step = 24
-    vals = []
+    vals, secs = [], []
     t_all = time.perf_counter()
     for it in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         r = cpu_baseline_prefill(xp, n_rows=rows_per_step)
         if it >= args.warmup:
             vals.append(r["value"])
+            secs.append(time.perf_counter() - t0)
     value = statistics.mean(vals)
-    sample = (f"per step {rows_per_step} evenly spaced query rows of the 128k full+select layer "
-              "in fp64, extrapolated to all rows by causal cost")
+    sample = (f"per step {rows_per_step} evenly spaced query rows of the {L}-token full+select "
+              "layer in fp64, extrapolated to all rows by causal cost")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2),
             "unit": "tokens/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")),
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(B * L / value * 1e3, 1), "higher_is_better": True,
+            # the measured time of one step's sample; `value` is extrapolated
+            # from it to the whole layer
+            "ms_per_step": round(statistics.mean(secs) * 1e3, 1),
+            "ms_per_step_extrapolated_full_layer": round(B * L / value * 1e3, 1),
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded planted-topic prefill)",
             "config": {"workload": f"{args.prefill} + {args.decode}", "L": L, "Hq": Hq, "d": d,
