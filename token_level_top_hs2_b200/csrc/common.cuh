@@ -55,6 +55,34 @@ HS2_DEV float ex2(float x) {
     return y;
 }
 
+// 2^x on the FMA pipe, for kernels whose exponentials outrun the MUFU pipe:
+// part of them go through this routine instead of ex2.
+//   * Cody and Waite's range reduction x = n + f, n an integer, |f| <= 1/2:
+//     adding 1.5 * 2^23 rounds x to an integer held in the low mantissa bits
+//     of the sum (exact for |x| < 2^22), and subtracting it back gives n as
+//     a float;
+//   * 2^f by a degree-5 polynomial (Horner, fused multiply-adds) whose
+//     coefficients were fitted here for least maximum relative error on
+//     [-1/2, 1/2] by Lawson's iteratively reweighted least squares; the
+//     fp32 evaluation stays within 2.2e-7 relative of 2^f;
+//   * 2^n enters by adding n to the exponent field of the result.
+// x is clamped to >= -125 so that the exponent cannot wrap: results below
+// 2^-125 come out as about 2^-125 instead of 0 (ex2.approx.ftz flushes
+// them); callers sum such values into much larger ones.
+HS2_DEV float ex2_fma(float x) {
+    const float xc = fmaxf(x, -125.f);
+    const float t = xc + 12582912.f;  // 1.5 * 2^23
+    const float n = t - 12582912.f;
+    const float f = xc - n;
+    float p = 1.32764713e-3f;
+    p = fmaf(p, f, 9.67554096e-3f);
+    p = fmaf(p, f, 5.55071309e-2f);
+    p = fmaf(p, f, 2.40221202e-1f);
+    p = fmaf(p, f, 6.93146944e-1f);
+    p = fmaf(p, f, 1.00000012e+0f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 HS2_DEV void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
