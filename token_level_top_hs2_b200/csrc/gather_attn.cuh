@@ -271,6 +271,14 @@ struct WarpAttn {
         }
     }
 
+    // Fragment order of the o accumulator: value i (0..4D/8-1) of lane L is
+    // o[i / 4][i % 4], i.e. row (L >> 2) + 8 * ((i >> 1) & 1) and column
+    // (2 * (L & 3) + (i & 1)) * (D / 8) + (i >> 2).  Storing value i of every
+    // lane at po[i * 32 + L] makes the 32 lanes of a store hit 32 banks.
+    HS2_DEV static int frag_row(int i, int L) { return (L >> 2) + 8 * ((i >> 1) & 1); }
+    HS2_DEV static int frag_col(int i, int L) { return (2 * (L & 3) + (i & 1)) * (D / 8) + (i >> 2); }
+    static constexpr int FRAG = NT * 4;  // values per lane
+
     // Write the unnormalised partial state (m, l, o) of rows < 16 into
     // shared/global arrays: pm[16], pl[16], po[16][D] (o in natural element order).
     HS2_DEV void dump(float* pm, float* pl, float* po) const {

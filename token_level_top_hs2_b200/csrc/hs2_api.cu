@@ -610,9 +610,11 @@ hs2_status run_decode_sparse(const hs2_decode_shape* s, const void* q, const voi
                              const void* vc, const float* ks, const float* vs,
                              const int32_t* lengths, const int32_t* idx, void* o,
                              cudaStream_t st, unsigned* flags) {
-    constexpr int WARPS = 6, CLUSTER = 8;
-    const size_t smem = (size_t)(WARPS + 1) * (16 * D + 32) * sizeof(float);
-    auto kern = decode_sparse_kernel<D, FP8, WARPS, CLUSTER>;
+    // two CTAs per SM where the registers allow it without spills (the bf16
+    // d = 128 tile needs more)
+    constexpr int WARPS = 6, CLUSTER = 8, MAXT = 1, MINB = (FP8 || D == 64) ? 2 : 1;
+    const size_t smem = (size_t)DecodeSparseSmem<D, FP8, WARPS, CLUSTER>::FLOATS * sizeof(float);
+    auto kern = decode_sparse_kernel<D, FP8, WARPS, CLUSTER, MAXT, MINB>;
     if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(s->B * CLUSTER);

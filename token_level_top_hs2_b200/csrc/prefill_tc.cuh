@@ -355,6 +355,11 @@ namespace tcfa {
 // The L x L score matrix never leaves the chip.
 constexpr int SBN = 256;   // keys per block
 constexpr int QSTAGE = 2;
+// Of every 16 exponentials of the score loop, this many run on the FMA pipe
+// (ex2_fma) and the rest on the MUFU pipe (ex2), which the loop otherwise
+// keeps busy with one operation per (key, head): 3 of 16 measured best at
+// 32k and 128k (2 and 4 within noise of it, 5 and 7 slower).
+constexpr int kSelFmaExp = 3;
 
 template <int D>
 struct Sel {
@@ -688,8 +693,10 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     tmem_ld16(s_lane + buf * SBN + c * 16, r);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; i++)
-                        acc[c * 16 + i] += ex2(fmaf(__uint_as_float(r[i]), scale2, -l2));
+                    for (int i = 0; i < 16; i++) {
+                        const float x = fmaf(__uint_as_float(r[i]), scale2, -l2);
+                        acc[c * 16 + i] += i < kSelFmaExp ? ex2_fma(x) : ex2(x);
+                    }
                 }
                 fence_before_sync();
                 __syncwarp();
