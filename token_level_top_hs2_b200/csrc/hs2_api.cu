@@ -229,7 +229,7 @@ bool map_kv(CUtensorMap* m, const void* x, int B, int L, int D, int rows) {
 }
 
 // ---------------------------------------------------------------- prefill
-// entries per (query row, key half) candidate stream
+// entries per (query row, key slice) candidate stream
 int pf_cap(int k) { return (int)round_up((size_t)2 * k + 128, 32); }
 
 struct PrefillWs {
@@ -243,7 +243,8 @@ PrefillWs prefill_ws(const hs2_prefill_shape* s) {
     w.fail_off = round_up(rows * s->Hq * sizeof(float), 256);
     w.fail_bytes = (size_t)s->B * ((s->L + tcfa::BM - 1) / tcfa::BM) * sizeof(unsigned);
     w.buf_off = round_up(w.fail_off + w.fail_bytes, 256);
-    w.total = w.buf_off + (s->k > 0 ? rows * 2 * pf_cap(s->k) * sizeof(uint64_t) : 0);
+    w.total = w.buf_off +
+              (s->k > 0 ? rows * tcfa::kSlices * pf_cap(s->k) * sizeof(uint64_t) : 0);
     return w;
 }
 
@@ -297,7 +298,7 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
             auto kb = tcfa::prefill_select_tc_kernel<D, true>;
             if (!set_smem(kb, smem)) return HS2_ERR_CUDA;
             float* mass = reinterpret_cast<float*>(ws + bw.mass_off);
-            kb<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k,
+            kb<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k,
                                                    s->W + s->k, 0, scale2, nullptr, idx, 0,
                                                    nullptr, nullptr, flags, mass, (int)bw.nblk);
             if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
@@ -315,10 +316,10 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
         if (cudaMemsetAsync(fail, 0, w.fail_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
         // speculative thresholds, then the exact selection for the query blocks
         // whose rows failed the check (a gated launch: the others return at once)
-        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
+        kern<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
                                       pf_cap(s->k), scale2, buf, idx, 1, nullptr, fail, flags, nullptr, 0);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
+        kern<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
                                       pf_cap(s->k), scale2, buf, idx, 0, fail, nullptr, flags, nullptr, 0);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }

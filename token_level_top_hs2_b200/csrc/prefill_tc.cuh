@@ -338,23 +338,33 @@ namespace tcfa {
 // streaming per-row top-k, for one block of 128 query rows and ALL heads.
 // For every 256-key block and every head h the MMA warp computes
 // S = Q_h K^T (M=128, N=256) into one of two TMEM buffers; Q_h tiles stream
-// through a 2-stage TMA ring, the K block through another.  Score warps
-// (thread = query row; warps 2-5 own keys 0..127 of the block, warps 6-9 keys
-// 128..255) add 2^(S*scale*log2e - lse2_h) into 128 registers; after the last
-// head they hold score(t, s) for their 128 keys and feed the candidates
-// (s <= t-W) into the (row, half) stream: keys >= the stream's threshold are
-// appended to its workspace buffer.  A buffer that would overflow is pruned
-// (one lane's buffer at a time) by a score-bit histogram.  A speculative prune
-// keeps only the keys reaching about 1.5 times the stream's expected share of
-// the row's top k, so the threshold approaches the row's final k-th score
-// early and few candidates are appended; if no bin boundary frees room, the
-// buffer is cut to about its k best (or exactly, by a radix select).  At the
-// end the two streams of a row are merged to exactly k, after an exact check
-// (at least min(k, candidates) keys reach the higher stream threshold); rows
-// that fail it flag their query block for a gated exact re-run.
+// through a 2-stage TMA ring, the K block through another.  Sixteen score
+// warps (thread = query row; four groups of four warps, group g owning keys
+// 64g..64g+63 of the block) add 2^(S*scale*log2e - lse2_h) into 64 registers;
+// after the last head they hold score(t, s) for their 64 keys and feed the
+// candidates (s <= t-W) into the (row, slice) stream: keys >= the stream's
+// threshold are appended to its workspace buffer.  A buffer that would
+// overflow is pruned (one lane's buffer at a time) by a score-bit histogram.
+// A speculative prune keeps only the keys reaching about 1.5 times the
+// stream's expected share of the row's top k, so the threshold approaches
+// the row's final k-th score early and few candidates are appended; if no bin
+// boundary frees room, the buffer is cut to about its k best (or exactly, by
+// a radix select).  At the end the four streams of a row are merged to
+// exactly k, after an exact check (at least min(k, candidates) keys reach the
+// highest stream threshold); rows that fail it flag their query block for a
+// gated exact re-run.
 // The L x L score matrix never leaves the chip.
 constexpr int SBN = 256;   // keys per block
 constexpr int QSTAGE = 2;
+// Score warps: 16, in four groups of four.  Group g owns keys 64g .. 64g+63 of
+// every 256-key block; within a group the four warps cover the four 32-lane
+// quarters of TMEM (a warp reaches lanes 32*(warp%4)..+31), i.e. the 128 query
+// rows.  Four score warps per SM sub-partition hide the latency of the TMEM
+// loads and of the candidate appends behind each other's exponentials.
+constexpr int kSlices = 4;
+constexpr int kSliceKeys = SBN / kSlices;          // 64
+constexpr int kScoreWarps = 4 * kSlices;           // 16
+constexpr int kSelThreads = 64 + 32 * kScoreWarps;  // + producer and MMA warps
 // Of every 16 exponentials of the score loop, this many run on the FMA pipe
 // (ex2_fma) and the rest on the MUFU pipe (ex2), which the loop otherwise
 // keeps busy with one operation per (key, head): 3 of 16 measured best at
@@ -368,14 +378,14 @@ struct Sel {
     static constexpr int DB = D / 64;
     static constexpr int OFF_K = 0;
     static constexpr int OFF_Q = 2 * KB;
-    static constexpr int OFF_HIST = OFF_Q + QSTAGE * QT;         // 8 warps x 260 ints
-    static constexpr int OFF_CNT = OFF_HIST + 8 * 260 * 4;       // [2][128] ints
-    static constexpr int OFF_TB = OFF_CNT + 2 * 128 * 4;         // [2][128] threshold bits
-    static constexpr int OFF_LSE = OFF_TB + 2 * 128 * 4;         // [16][128] floats
+    static constexpr int OFF_HIST = OFF_Q + QSTAGE * QT;                 // score warps x 260 ints
+    static constexpr int OFF_CNT = OFF_HIST + kScoreWarps * 260 * 4;     // [kSlices][128] ints
+    static constexpr int OFF_TB = OFF_CNT + kSlices * 128 * 4;           // [kSlices][128] bits
+    static constexpr int OFF_LSE = OFF_TB + kSlices * 128 * 4;           // [16][128] floats
     static constexpr int SMEM = OFF_LSE + 16 * 128 * 4 + 1024;
-    // final selection reuses the K region: per warp a boundary-bin buffer
-    static constexpr int BCAP = 1024;
-    static_assert(8 * BCAP * 8 <= 2 * KB, "boundary buffers must fit the K region");
+    // final selection reuses the K region: per score warp a boundary-bin buffer
+    static constexpr int BCAP = 2 * KB / (kScoreWarps * 8);
+    static_assert(kScoreWarps * BCAP * 8 <= 2 * KB, "boundary buffers must fit the K region");
 };
 
 struct SelBars {
@@ -481,14 +491,14 @@ HS2_DEV uint64_t warp_cut(uint64_t* buf, int cnt, int k, int* hist) {
     return thr;
 }
 
-// grid (ceil(L/128), B), 320 threads.  wsbuf: [B*L][2][cap] keys.
+// grid (ceil(L/128), B), kSelThreads threads.  wsbuf: [B*L][kSlices][cap] keys.
 // BLK (the block-level selector of HySparse, the predecessor the HySparse2
 // summary ablates against in "Limits"): instead of streaming token
 // candidates, every score thread writes the attention mass of the 64-key
 // blocks it holds -- the sum of its candidates' scores -- to
 // mass[b*L + t][nblk]; block_select_kernel picks the blocks.
 template <int D, bool BLK = false>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kSelThreads, 1)
 prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                          const __grid_constant__ CUtensorMap map_k,
                          const float* __restrict__ lse, int L, int Hq, int W, int kk, int S,
@@ -519,7 +529,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             mbar_init(&bars.k_full[i], 1);
             mbar_init(&bars.k_empty[i], 1);
             mbar_init(&bars.s_full[i], 1);
-            mbar_init(&bars.s_empty[i], 8);
+            mbar_init(&bars.s_empty[i], kScoreWarps);
         }
         for (int i = 0; i < QSTAGE; i++) {
             mbar_init(&bars.q_full[i], 1);
@@ -605,22 +615,24 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         }
     } else {
         // ---------------------------------------------------------- scores
-        const int half = (warp - 2) >> 2;        // keys half*128 .. +127 of each block
+        const int slice = (warp - 2) >> 2;      // keys slice*64 .. +63 of each block
         const int row = (warp & 3) * 32 + lane;  // TMEM lane
         const int t = qb * BM + row;
         const bool valid = t < L;
         const int maxkey = t - W;                // candidates 0..maxkey
-        const uint32_t s_lane = tmem + ((uint32_t)((warp & 3) * 32) << 16) + half * 128;
+        const uint32_t s_lane =
+            tmem + ((uint32_t)((warp & 3) * 32) << 16) + slice * kSliceKeys;
         int* hist = reinterpret_cast<int*>(smem + F::OFF_HIST) + (warp - 2) * 260;
-        uint64_t* my_buf = wsbuf + (((size_t)b * L + (valid ? t : 0)) * 2 + half) * cap;
+        uint64_t* my_buf =
+            wsbuf + (((size_t)b * L + (valid ? t : 0)) * kSlices + slice) * cap;
         // log2-domain lse of this row per head, in shared memory: [h][row]
         float* lse2 = reinterpret_cast<float*>(smem + F::OFF_LSE);
-        if (half == 0)
+        if (slice == 0)
             for (int h = 0; h < 16; h++)
                 lse2[h * 128 + row] = (valid && h < Hq)
                                           ? __ldg(lse + ((size_t)b * L + t) * Hq + h) * kLog2e
                                           : INFINITY;
-        asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 score warps
+        asm volatile("bar.sync 1, %0;" ::"r"(32 * kScoreWarps) : "memory");  // score warps
         int cnt = 0;
         uint32_t thr_bits = 0;  // appended keys have score bits >= thr_bits
         // histogram origin of a stream's first prune: 1/64 of the row's mean
@@ -628,21 +640,22 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         const uint32_t base_bits = __float_as_uint((float)Hq / (64.f * (float)(t + 1)));
         bool ok = true;
         for (int kb = 0; kb < n_kb && ok; kb++) {
-            const int key0 = kb * SBN + half * 128;
+            const int key0 = kb * SBN + slice * kSliceKeys;
             const bool streams = valid && key0 <= maxkey;
             if constexpr (!BLK) {
-                // the stream has seen kb*128 of the row's n_row candidates and
+                // the stream has seen kb*64 of the row's n_row candidates and
                 // buffers every one of them at or above its threshold; a
                 // speculative prune keeps 1.5 times their expected share of
                 // the row's top k, plus 32 (on the planted-topic workloads no
                 // row failed the exact check at this margin; at 1.25x + 16 a
                 // few did).  It runs when the buffer is full, and early, as
-                // soon as it holds twice that share plus 256, so the threshold
+                // soon as it holds twice that share plus 128, so the threshold
                 // rises long before the first 2k candidates are buffered.
-                const long long r_own = 3LL * kk * (kb * 128) / (2LL * max(maxkey + 1, 1)) + 32;
-                const bool full = cnt + 128 > cap;
-                const bool early = speculate && r_own < kk && cnt >= 2 * r_own + 256;
-                // make room for this block's 128 candidates before accumulating
+                const long long r_own =
+                    3LL * kk * (kb * kSliceKeys) / (2LL * max(maxkey + 1, 1)) + 32;
+                const bool full = cnt + kSliceKeys > cap;
+                const bool early = speculate && r_own < kk && cnt >= 2 * r_own + 128;
+                // make room for this block's candidates before accumulating
                 unsigned need = __ballot_sync(0xffffffffu, streams && (full || early));
                 while (need) {
                     const int src = __ffs(need) - 1;
@@ -661,10 +674,11 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         // a full buffer is pruned to k below, an early one is
                         // left as it was)
                         if (r < kk)
-                            ncnt = warp_prune(sbuf, scnt, (int)r, cap - 128, sbase, hist, &ntb);
+                            ncnt = warp_prune(sbuf, scnt, (int)r, cap - kSliceKeys, sbase, hist,
+                                              &ntb);
                     }
                     if (ncnt < 0 && sfull)
-                        ncnt = warp_prune(sbuf, scnt, kk, cap - 128, sbase, hist, &ntb);
+                        ncnt = warp_prune(sbuf, scnt, kk, cap - kSliceKeys, sbase, hist, &ntb);
                     if (ncnt < 0 && sfull) {  // no histogram boundary frees room: exact cut to k
                         const uint64_t nthr = warp_cut(sbuf, scnt, kk, hist);
                         ntb = (uint32_t)(nthr >> 32);
@@ -676,9 +690,9 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                     }
                 }
             }
-            float acc[128];
+            float acc[kSliceKeys];
 #pragma unroll
-            for (int i = 0; i < 128; i++) acc[i] = 0.f;
+            for (int i = 0; i < kSliceKeys; i++) acc[i] = 0.f;
             for (int h = 0; h < Hq; h++) {
                 const int it = kb * Hq + h, buf = it & 1;
                 if (!mbar_wait(&bars.s_full[buf], (it >> 1) & 1, abort_, flags)) {
@@ -688,7 +702,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 fence_after_sync();
                 const float l2 = lse2[h * 128 + row];
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
+                for (int c = 0; c < kSliceKeys / 16; c++) {
                     uint32_t r[16];
                     tmem_ld16(s_lane + buf * SBN + c * 16, r);
                     tmem_ld_wait();
@@ -704,35 +718,30 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             if (!ok) break;
             if constexpr (BLK) {
-                // ---- all heads summed: the mass of each 64-key block with a
-                // candidate (eight partial sums of eight, then a tree)
+                // ---- all heads summed: the mass of this thread's 64-key block
+                // (its candidates only; eight partial sums of eight, then a tree)
                 if (streams) {
+                    float p8[8];
 #pragma unroll
-                    for (int u = 0; u < 2; u++) {
-                        const int bk0 = key0 + 64 * u;
-                        if (bk0 > maxkey) break;
-                        float p8[8];
+                    for (int g = 0; g < 8; g++) {
+                        float a = 0.f;
 #pragma unroll
-                        for (int g = 0; g < 8; g++) {
-                            float a = 0.f;
-#pragma unroll
-                            for (int i = 0; i < 8; i++) {
-                                const int j = 64 * u + 8 * g + i;
-                                a += (key0 + j <= maxkey) ? acc[j] : 0.f;
-                            }
-                            p8[g] = a;
+                        for (int i = 0; i < 8; i++) {
+                            const int j = 8 * g + i;
+                            a += (key0 + j <= maxkey) ? acc[j] : 0.f;
                         }
-                        const float m = ((p8[0] + p8[1]) + (p8[2] + p8[3])) +
-                                        ((p8[4] + p8[5]) + (p8[6] + p8[7]));
-                        mass[((size_t)b * L + t) * nblk + bk0 / 64] = m;
+                        p8[g] = a;
                     }
+                    const float m = ((p8[0] + p8[1]) + (p8[2] + p8[3])) +
+                                    ((p8[4] + p8[5]) + (p8[6] + p8[7]));
+                    mass[((size_t)b * L + t) * nblk + key0 / kSliceKeys] = m;
                 }
                 continue;
             }
             // ---- all heads summed: stream the block's candidates
             if (streams) {
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
+                for (int c = 0; c < kSliceKeys / 16; c++) {
 #pragma unroll
                     for (int i = 0; i < 16; i++) {
                         const int j = c * 16 + i;
@@ -748,8 +757,8 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
             }
         }
-        cnts[half * 128 + row] = cnt;
-        tbs[half * 128 + row] = thr_bits;
+        cnts[slice * 128 + row] = cnt;
+        tbs[slice * 128 + row] = thr_bits;
     }
     fence_before_sync();
     __syncthreads();
@@ -761,28 +770,38 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         return;
     }
     // ---------------------------------------------- final selection per row
-    // Warps 2..9: warp w takes rows w-2, w+6, ... (16 rows each).  The union of
-    // a row's two streams is histogrammed relative to the higher stream
+    // Score warp w (0..15) takes rows w, w+16, ... (8 rows each).  The union of
+    // a row's kSlices streams is histogrammed relative to the highest stream
     // threshold; keys above the boundary bin are written at once, the boundary
     // bin is gathered into shared memory (the freed K region) and cut exactly
     // there, so that exactly kk globals follow the window.
     if (warp >= 2 && !*abort_) {
         int* hist = reinterpret_cast<int*>(smem + F::OFF_HIST) + (warp - 2) * 260;
         uint64_t* bnd = reinterpret_cast<uint64_t*>(smem + F::OFF_K) + (warp - 2) * F::BCAP;
-        for (int row = warp - 2; row < BM; row += 8) {
+        for (int row = warp - 2; row < BM; row += kScoreWarps) {
             const int t = qb * BM + row;
             if (t >= L) break;
-            const int n0 = cnts[row], n1 = cnts[128 + row];
-            const uint64_t* b0 = wsbuf + (((size_t)b * L + t) * 2 + 0) * cap;
-            const uint64_t* b1 = wsbuf + (((size_t)b * L + t) * 2 + 1) * cap;
-            auto get = [&](int i) { return i < n0 ? __ldcg(b0 + i) : __ldcg(b1 + (i - n0)); };
-            const int n = n0 + n1;
+            // the streams' counts as running offsets into the union
+            int off[kSlices + 1];
+            off[0] = 0;
+#pragma unroll
+            for (int q = 0; q < kSlices; q++) off[q + 1] = off[q] + cnts[q * 128 + row];
+            const uint64_t* rb = wsbuf + ((size_t)b * L + t) * kSlices * cap;
+            auto get = [&](int i) {
+                int q = 0;
+#pragma unroll
+                for (int u = 1; u < kSlices; u++) q += i >= off[u];
+                return __ldcg(rb + (size_t)q * cap + (i - off[q]));
+            };
+            const int n = off[kSlices];
             const int w0 = max(0, t - W + 1);
             const int wl = t - w0 + 1;
             int32_t* out = idx + ((size_t)b * L + t) * S;
             for (int i = lane; i < wl; i += 32) out[i] = w0 + i;
             int wp = wl;
-            const uint32_t base = max(tbs[row], tbs[128 + row]);
+            uint32_t base = tbs[row];
+#pragma unroll
+            for (int q = 1; q < kSlices; q++) base = max(base, tbs[q * 128 + row]);
             if (speculate) {
                 // every key whose score bits reach `base` is in the union; the
                 // row is exact iff at least min(k, candidates) of them are
@@ -901,6 +920,7 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
 // candidate positions of the chosen blocks (in block order), then -1.
 constexpr int kBlkWarps = 4;
 constexpr int kBlock = 64;
+static_assert(kBlock == kSliceKeys, "a score thread's key slice is one selector block");
 
 __global__ void __launch_bounds__(kBlkWarps * 32)
 block_select_kernel(const float* __restrict__ mass, int B, int L, int W, int nsel, int S,
