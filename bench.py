@@ -452,6 +452,33 @@ def run_ours(args, world, rank, local):
     assert hs2.hs2_get_last_device_error() == 0
     n_launch = (launches(pf) + launches(dc) + 1 + 3) * args.steps
 
+    # worst case of the full layer: the same queries and keys with key
+    # relevance falling along the sequence (early keys score higher), so the
+    # selection's speculative stream thresholds fail on many query blocks and
+    # their gated exact re-run does the work again
+    worst = None
+    if not args.no_configs:
+        g = torch.Generator(device="cpu").manual_seed(32)
+        u = torch.randn(d, generator=g)
+        u = (u / u.norm()).to(dev)
+        ramp = 6.0 * (1.0 - torch.arange(L, dtype=torch.float32, device=dev) / L)
+        kw = (pf.k.float() + ramp[None, :, None] * u).bfloat16()
+        qw = (pf.q.float() + 3.0 * u).bfloat16()
+        del ramp
+
+        def full_worst():
+            hs2.hs2_full_attn_select(qw, kw, pf.v, W, K, o=pf.o, lse=pf.lse, idx=pf.idx,
+                                     workspace=pf.ws)
+        for _ in range(args.warmup):
+            full_worst()
+        torch.cuda.synchronize()
+        time_pieces([("full_select_decaying_keys", full_worst)], args.steps, flush, stream, times)
+        n_launch += full_launches * args.steps
+        nqb = (L + 127) // 128
+        fail_off = (B * L * Hq * 4 + 255) // 256 * 256
+        worst = int(pf.ws[fail_off: fail_off + 4 * B * nqb].view(torch.int32).sum().item())
+        del qw, kw
+
     # the other workloads: warm-up, then the same number of timed repetitions
     for w in others:
         if isinstance(w, DecodeWork):
@@ -504,6 +531,15 @@ def run_ours(args, world, rank, local):
                 "n_sparse_layers": len(w.qs)}
 
     cfg = {pf.name: prefill_summary(pf), dc.name: decode_summary(dc)}
+    if worst is not None:
+        t_w = ms["full_select_decaying_keys"] / 1e3
+        cfg[pf.name]["full_select_decaying_keys_ms"] = round(t_w * 1e3, 4)
+        cfg[pf.name]["full_select_decaying_keys_tok_s"] = round(world * B * L / t_w, 1)
+        cfg[pf.name]["full_select_decaying_keys_failed_query_blocks"] = worst
+        cfg[pf.name]["full_select_decaying_keys_note"] = (
+            "worst case: key relevance falling along the sequence (+6u ramp on keys, +3u on "
+            "queries) defeats the speculative stream thresholds; the failed query blocks are "
+            "recomputed by the gated exact re-run")
     for w in others:
         cfg[w.name] = (prefill_summary(w, w.name + "/") if isinstance(w, PrefillWork)
                        else decode_summary(w, w.name + "/"))

@@ -88,8 +88,9 @@ int hs2_version(void);
 
 /*
  * Bytes of device workspace hs2_full_attn_select needs for `shape`
- * (0 for an invalid shape).  Per query row it holds a candidate buffer of
- * 2k+256 (score, position) entries plus the row's running threshold and count.
+ * (0 for an invalid shape): the lse (when the caller passes none), one flag
+ * word per 128-row query block, and per query row four candidate streams of
+ * round_up(2k+128, 32) 8-byte (score, position) keys.
  */
 size_t hs2_full_attn_select_workspace(const hs2_prefill_shape* shape);
 

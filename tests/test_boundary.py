@@ -51,8 +51,11 @@ def test_status_strings(lib):
 def test_workspace_sizes(lib):
     s = hs2.prefill_shape(1, 131072, 16, 128, 128, 1024)
     ws = hs2.hs2_full_attn_select_workspace(s)
-    # lse area + one (2k+256)-entry buffer of 8-byte keys per query row
-    assert ws >= 131072 * (2 * 1024 + 256) * 8
+    # lse area, the query-block flags, and four candidate streams of
+    # round_up(2k + 128, 32) 8-byte keys per query row
+    cap = (2 * 1024 + 128 + 31) // 32 * 32
+    assert ws >= 131072 * 4 * cap * 8 + 131072 * 16 * 4
+    assert ws < 131072 * 4 * cap * 8 + 131072 * 16 * 4 + 4096 + 1024 * 4
     assert hs2.hs2_full_attn_select_workspace(hs2.prefill_shape(1, 10, 3, 128, 8, 8)) == 0
     d = hs2.decode_shape(16, 262144, 16, 128, 128, 1024)
     assert hs2.hs2_decode_select_workspace(d) > 16 * 1024 * 8
