@@ -58,6 +58,8 @@ def parse():
     p.add_argument("--no-clocks", action="store_true")
     p.add_argument("--no-configs", action="store_true",
                    help="skip the other workloads measured after the timed step")
+    p.add_argument("--once", action="store_true",
+                   help="call each bench kernel once on the workloads, untimed (for profilers)")
     return p.parse_args()
 
 
@@ -385,6 +387,28 @@ def run_ours(args, world, rank, local):
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    if args.once:
+        # one call of each bench entry point on the workloads, untimed (for
+        # profilers), in a fixed order: full+select (pass 1, selection, gated
+        # re-run), a sparse layer, decode select (zeroing, pass 1, sketch
+        # score, sketch gather, gated fallbacks), a decode sparse layer, a
+        # second full layer with the first sparse layer's queries and the
+        # overlap of the two selections, the block-level selector
+        pf.full()
+        pf.sparse(0)
+        dc.select()
+        dc.sparse(0)
+        own = torch.empty_like(pf.idx)
+        hs2.hs2_full_attn_select(pf.qs[0], pf.k, pf.v, W, K, o=pf.os_, lse=pf.lse, idx=own,
+                                 workspace=pf.ws)
+        hs2.hs2_selection_overlap(pf.idx, own, W, K)
+        hs2.hs2_full_attn_select_blocks(pf.q, pf.k, pf.v, W, K, o=pf.o, lse=pf.lse)
+        torch.cuda.synchronize()
+        assert hs2.hs2_get_last_device_error() == 0
+        if rank == 0:
+            print("once: ok", flush=True)
+        return
+
     # cross-layer overlap (diagnostic): the inherited selection against the one
     # the first sparse layer's own queries give, made once outside the timing
     idx_own = torch.empty_like(pf.idx)
@@ -621,9 +645,27 @@ def run_ours(args, world, rank, local):
         print(json.dumps(line), flush=True)
 
 
+def e2e_chunks(L, n_sms=148, bm=128):
+    """Query-row chunks of the end-to-end pipeline.  Full layer: a first
+    quarter (compute starts once it and its K/V rows are in), a second
+    quarter, then the rest.  Selection: everything but the last wave of query
+    blocks (n_sms blocks, the heaviest), then that wave, so that only its
+    indices remain to be copied out after the last kernel."""
+    def cut(x):
+        return max(bm, min(L, (int(x) // bm) * bm))
+    attn = sorted({0, cut(L / 4), cut(L / 2), L})
+    last = L - n_sms * bm
+    sel = [0, last, L] if last >= bm else [0, L]
+    return attn, sel
+
+
 def e2e_prefill(hs2, xp, args, world, dev, W, K, ws, flush):
-    """Prefill full+select through the public call with host buffers: pinned
-    host Q/K/V -> device, the call, O and idx -> pinned host, all timed."""
+    """Prefill full+select through the public calls with host buffers: Q, K, V
+    copied in from pinned host memory, O and idx copied back, all timed.  The
+    copies overlap the kernels: the full layer runs on query-row chunks
+    (hs2_full_attn_rows) as their rows arrive, O chunks go back while later
+    work runs, and the selection (hs2_select_rows) runs in two chunks with the
+    first chunk's indices copied out during the second."""
     B, L, Hq, d = xp.q.shape
     hq, hk, hv = xp.q.pin_memory(), xp.k_.pin_memory(), xp.v.pin_memory()
     ho = torch.empty_like(hq).pin_memory()
@@ -635,26 +677,39 @@ def e2e_prefill(hs2, xp, args, world, dev, W, K, ws, flush):
     idx = torch.empty(B, L, W + K, dtype=torch.int32, device=dev)
     lse = torch.empty(B, L, Hq, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    side = torch.cuda.Stream()
+    cin, cout = torch.cuda.Stream(), torch.cuda.Stream()
+    attn, sel = e2e_chunks(L)
     ts = []
     for it in range(args.warmup + args.steps):
         flush.zero_()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        o_ready = torch.cuda.Event()
         e0.record(stream)
-        q.copy_(hq, non_blocking=True)
-        k.copy_(hk, non_blocking=True)
-        v.copy_(hv, non_blocking=True)
-        # O is final after the attention half: its copy to the host runs on a
-        # second stream while the selection computes
-        hs2.hs2_full_attn(q, k, v, W=W, k_top=K, o=o, lse=lse)
-        o_ready.record(stream)
-        side.wait_event(o_ready)
-        with torch.cuda.stream(side):
-            ho.copy_(o, non_blocking=True)
-        hs2.hs2_select(q, k, lse, W, K, idx=idx, workspace=ws)
-        hidx.copy_(idx, non_blocking=True)
-        stream.wait_stream(side)
+        cin.wait_stream(stream)
+        cout.wait_stream(stream)
+        arrived = []
+        with torch.cuda.stream(cin):
+            for a, b in zip(attn[:-1], attn[1:]):
+                for dst, src in ((k, hk), (v, hv), (q, hq)):
+                    dst[:, a:b].copy_(src[:, a:b], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(cin)
+                arrived.append(ev)
+        for (a, b), ev in zip(zip(attn[:-1], attn[1:]), arrived):
+            stream.wait_event(ev)
+            hs2.hs2_full_attn_rows(q, k, v, a, b, o=o, lse=lse, W=W, k_top=K)
+            done = torch.cuda.Event()
+            done.record(stream)
+            cout.wait_event(done)
+            with torch.cuda.stream(cout):
+                ho[:, a:b].copy_(o[:, a:b], non_blocking=True)
+        for a, b in zip(sel[:-1], sel[1:]):
+            hs2.hs2_select_rows(q, k, lse, W, K, a, b, idx=idx, workspace=ws)
+            done = torch.cuda.Event()
+            done.record(stream)
+            cout.wait_event(done)
+            with torch.cuda.stream(cout):
+                hidx[:, a:b].copy_(idx[:, a:b], non_blocking=True)
+        stream.wait_stream(cout)
         e1.record(stream)
         torch.cuda.synchronize()
         if it >= args.warmup:
@@ -664,8 +719,10 @@ def e2e_prefill(hs2, xp, args, world, dev, W, K, ws, flush):
     d2h = ho.numel() * ho.element_size() + hidx.numel() * hidx.element_size()
     return {"value": round(world * B * L / t, 1), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "what": "prefill full+select at 128k: pinned H2D of q,k,v, hs2_full_attn, then "
-                    "hs2_select while O is copied to the host on a second stream, D2H of idx"}
+            "what": f"prefill full+select at {L} tokens from pinned host buffers: q,k,v copied in "
+                    f"by query-row chunks {attn} while hs2_full_attn_rows runs on the chunks "
+                    f"already in, O copied back per chunk, hs2_select_rows on chunks {sel} with "
+                    "the first chunk's idx copied back during the second"}
 
 
 def cores_used():

@@ -132,6 +132,26 @@ hs2_status hs2_select(const hs2_prefill_shape* shape, const void* q, const void*
                       hs2_stream_t stream);
 
 /*
+ * hs2_full_attn and hs2_select for the query rows [row0, row1) of every
+ * sequence only (same "What differs" computation, restricted to those rows):
+ * row0 a multiple of 128, row1 a multiple of 128 or L, 0 <= row0 < row1 <= L.
+ * A query row t reads only K/V rows 0..t, so these calls read K and V rows
+ * 0..row1-1, q rows [row0, row1) and (hs2_select_rows) lse rows [row0, row1),
+ * and write o, lse or idx rows [row0, row1) only; the tensors keep their
+ * full [B, L, ...] shapes.  Results equal those rows of the full calls.  A
+ * caller streaming a long prompt in can run the rows that have arrived while
+ * the rest is still being copied, and copy finished rows out while later ones
+ * compute.  The same workspace size as hs2_full_attn_select; calls on one
+ * workspace must not overlap in time.
+ */
+hs2_status hs2_full_attn_rows(const hs2_prefill_shape* shape, int row0, int row1, const void* q,
+                              const void* k, const void* v, void* o, float* lse,
+                              hs2_stream_t stream);
+hs2_status hs2_select_rows(const hs2_prefill_shape* shape, int row0, int row1, const void* q,
+                           const void* k, const float* lse, int32_t* idx, void* workspace,
+                           size_t workspace_bytes, hs2_stream_t stream);
+
+/*
  * Block-level selector variant: the full layer of HySparse, the predecessor
  * the HySparse2 summary compares against ("Limits": 64-token blocks, 1,024
  * global tokens, a separate 128-token local window).  Same exact attention

@@ -93,3 +93,17 @@ def test_source_hash_covers_every_kernel_source():
     h = bench.csrc_hash()
     assert len(h) == 16 and int(h, 16) >= 0
     assert h == bench.csrc_hash()  # deterministic
+
+
+def test_e2e_chunks_are_valid_row_ranges():
+    # the row-range calls need chunk starts on 128-row query blocks and ends on
+    # a block boundary or at L; the chunks tile [0, L)
+    for L in (131072, 32768, 1024, 1000, 300):
+        attn, sel = bench.e2e_chunks(L)
+        for cuts in (attn, sel):
+            assert cuts[0] == 0 and cuts[-1] == L
+            assert all(a < b for a, b in zip(cuts[:-1], cuts[1:]))
+            assert all(c % 128 == 0 for c in cuts[:-1])
+    attn, sel = bench.e2e_chunks(131072)
+    assert attn == [0, 32768, 65536, 131072]
+    assert sel == [0, 131072 - 148 * 128, 131072]  # the last wave of query blocks

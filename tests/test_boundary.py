@@ -216,3 +216,15 @@ def test_bounded_wait_check_rejects_bad_limits(lib):
     # refused before anything is launched (no GPU is touched)
     assert lib.hs2_check_bounded_wait(0, None) == hs2.HS2_ERR_INVALID_ARG
     assert lib.hs2_check_bounded_wait(1000001, None) == hs2.HS2_ERR_INVALID_ARG
+
+
+def test_row_range_calls_reject_bad_ranges(lib):
+    s = hs2.prefill_shape(1, 1000, 16, 128, 8, 8)
+    for r0, r1 in [(-128, 128), (0, 0), (256, 128), (1, 128), (0, 100), (0, 1001), (128, 999)]:
+        assert lib.hs2_full_attn_rows(ctypes.byref(s), r0, r1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                      None) == hs2.HS2_ERR_INVALID_ARG, (r0, r1)
+        assert lib.hs2_select_rows(ctypes.byref(s), r0, r1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                   1 << 40, None) == hs2.HS2_ERR_INVALID_ARG, (r0, r1)
+    # a range ending at L need not end on a 128-row boundary
+    assert lib.hs2_select_rows(ctypes.byref(s), 896, 1000, FAKE, FAKE, FAKE, FAKE, FAKE, 16,
+                               None) == hs2.HS2_ERR_WORKSPACE

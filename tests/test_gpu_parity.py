@@ -631,6 +631,36 @@ def test_split_full_attn_and_select_equal_the_combined_call(cuda_lib):
     assert torch.equal(torch.sort(idx, dim=-1).values, torch.sort(idx2, dim=-1).values)
 
 
+def test_row_range_calls_equal_the_full_layer(cuda_lib):
+    """The full layer in query-row chunks (each chunk reads only the K/V rows
+    it needs) gives the whole call's O and lse bit for bit and the same
+    selections."""
+    x = inputs.make_prefill(2, 1000, 16, 128, 64, 256, n_topics=8, seg=256,
+                            seed=inputs.seed_for(0, 6))
+    B, L, Hq, d = x.q.shape
+    q, k, v = cuda(x.q), cuda(x.k_), cuda(x.v)
+    o, lse, idx = cuda_lib.hs2_full_attn_select(q, k, v, x.W, x.k)
+    o2, lse2 = torch.full_like(o, 7.0), torch.full_like(lse, 7.0)
+    idx2 = torch.full_like(idx, -7)
+    ws = torch.empty(cuda_lib.hs2_full_attn_select_workspace(
+        cuda_lib.prefill_shape(B, L, Hq, d, x.W, x.k)), dtype=torch.uint8, device="cuda")
+    cuts = [0, 128, 384, 512, 1000]
+    for r0, r1 in zip(cuts[:-1], cuts[1:]):
+        cuda_lib.hs2_full_attn_rows(q, k, v, r0, r1, o=o2, lse=lse2)
+    for r0, r1 in zip(cuts[:-1], cuts[1:]):
+        cuda_lib.hs2_select_rows(q, k, lse2, x.W, x.k, r0, r1, idx=idx2, workspace=ws)
+    torch.cuda.synchronize()
+    assert cuda_lib.hs2_get_last_device_error() == 0
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    assert torch.equal(torch.sort(idx, dim=-1).values, torch.sort(idx2, dim=-1).values)
+    # a chunk writes only its own rows
+    o3 = torch.full_like(o, 7.0)
+    cuda_lib.hs2_full_attn_rows(q, k, v, 128, 384, o=o3, lse=lse2)
+    torch.cuda.synchronize()
+    assert torch.equal(o3[:, 128:384], o[:, 128:384])
+    assert bool((o3[:, :128] == 7.0).all()) and bool((o3[:, 384:] == 7.0).all())
+
+
 # ------------------------------------------------ the largest index rows
 # W + k = 2048, the largest selection the library accepts.
 

@@ -40,7 +40,8 @@ EXPORTED = [
     "hs2_decode_select_noalloc", "hs2_selection_overlap",
     "hs2_full_attn_select_blocks_workspace", "hs2_full_attn_select_blocks",
     "hs2_decode_stage_workspace", "hs2_decode_stage", "hs2_decode_sparse_staged",
-    "hs2_full_attn", "hs2_select", "hs2_check_bounded_wait",
+    "hs2_full_attn", "hs2_select", "hs2_check_bounded_wait", "hs2_full_attn_rows",
+    "hs2_select_rows",
 ]
 
 
@@ -88,6 +89,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     L.hs2_full_attn.restype = i32
     L.hs2_select.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
     L.hs2_select.restype = i32
+    L.hs2_full_attn_rows.argtypes = [P, i32, i32, vp, vp, vp, vp, vp, vp]
+    L.hs2_full_attn_rows.restype = i32
+    L.hs2_select_rows.argtypes = [P, i32, i32, vp, vp, vp, vp, vp, sz, vp]
+    L.hs2_select_rows.restype = i32
     L.hs2_full_attn_select_blocks_workspace.argtypes = [P, i32]
     L.hs2_full_attn_select_blocks_workspace.restype = sz
     L.hs2_full_attn_select_blocks.argtypes = [P, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -263,6 +268,36 @@ def hs2_select(q, k, lse, W: int, k_top: int, *, scale=None, idx=None, workspace
                            _ptr(workspace, "workspace"),
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "hs2_select")
+    return idx
+
+
+def hs2_full_attn_rows(q, k, v, row0: int, row1: int, *, o, lse, W: int = 1, k_top: int = 0,
+                       scale=None, stream=None):
+    """hs2_full_attn for query rows [row0, row1) of every sequence, into the
+    full-size o [B,L,Hq,d] and lse [B,L,Hq]; reads K/V rows 0..row1-1."""
+    B, L, Hq, d = q.shape
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    n, nh = B * L * d, B * L * Hq
+    st = load().hs2_full_attn_rows(ctypes.byref(shape), row0, row1, _ptr(q, "q", _BF16),
+                                   _ptr(k, "k", _BF16, n), _ptr(v, "v", _BF16, n),
+                                   _ptr(o, "o", _BF16, nh * d), _ptr(lse, "lse", _F32, nh),
+                                   _stream(stream))
+    _check(st, "hs2_full_attn_rows")
+    return o, lse
+
+
+def hs2_select_rows(q, k, lse, W: int, k_top: int, row0: int, row1: int, *, idx, workspace,
+                    scale=None, stream=None):
+    """hs2_select for query rows [row0, row1) of every sequence, into the
+    full-size idx [B,L,W+k]."""
+    B, L, Hq, d = q.shape
+    shape = prefill_shape(B, L, Hq, d, W, k_top, scale)
+    st = load().hs2_select_rows(ctypes.byref(shape), row0, row1, _ptr(q, "q", _BF16),
+                                _ptr(k, "k", _BF16, B * L * d), _ptr(lse, "lse", _F32, B * L * Hq),
+                                _ptr(idx, "idx", _I32, B * L * (W + k_top)),
+                                _ptr(workspace, "workspace"),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "hs2_select_rows")
     return idx
 
 

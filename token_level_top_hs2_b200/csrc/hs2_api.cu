@@ -267,8 +267,11 @@ template <int D>
 hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void* k,
                            const void* v, void* o, float* lse, int32_t* idx, uint8_t* ws,
                            cudaStream_t st, unsigned* flags, bool blocks = false,
-                           int phases = 3) {
-    // phases: 1 = exact attention (O, lse), 2 = the selection from lse
+                           int phases = 3, int row0 = 0, int row1 = -1) {
+    // phases: 1 = exact attention (O, lse), 2 = the selection from lse;
+    // query rows [row0, row1) of every sequence (row0 a multiple of 128)
+    if (row1 < 0) row1 = s->L;
+    const int qb0 = row0 / tcfa::BM, qb1 = (row1 + tcfa::BM - 1) / tcfa::BM;
     const PrefillWs w = prefill_ws(s);
     const BlockWs bw = block_ws(s);  // same lse area (offset 0) as the token path
     float* lse_p = lse ? lse : reinterpret_cast<float*>(ws + w.lse_off);
@@ -281,9 +284,9 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
         const size_t smem = tcfa::Fwd<D>::SMEM;
         auto kern = tcfa::prefill_fwd_tc_kernel<D>;
         if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
-        dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->Hq / 2, s->B);
-        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse_p, s->L,
-                                      s->Hq, scale2, flags);
+        dim3 grid(qb1 - qb0, s->Hq / 2, s->B);
+        kern<<<grid, tcfa::kThreads, smem, st>>>(mq, mk, mv, static_cast<__nv_bfloat16*>(o), lse_p,
+                                                 s->L, qb1, s->Hq, scale2, flags);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     if (phases & 2) {
@@ -292,13 +295,13 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
             !map_kv(&mk, k, s->B, s->L, D, tcfa::SBN))
             return HS2_ERR_CUDA;
         const size_t smem = tcfa::Sel<D>::SMEM;
-        dim3 grid((s->L + tcfa::BM - 1) / tcfa::BM, s->B);
+        dim3 grid(qb1 - qb0, s->B);
         if (blocks) {
             // block masses, then the choice of blocks per row
             auto kb = tcfa::prefill_select_tc_kernel<D, true>;
             if (!set_smem(kb, smem)) return HS2_ERR_CUDA;
             float* mass = reinterpret_cast<float*>(ws + bw.mass_off);
-            kb<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k,
+            kb<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, qb1, s->Hq, s->W, s->k,
                                                    s->W + s->k, 0, scale2, nullptr, idx, 0,
                                                    nullptr, nullptr, flags, mass, (int)bw.nblk);
             if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
@@ -316,11 +319,13 @@ hs2_status run_full_select(const hs2_prefill_shape* s, const void* q, const void
         if (cudaMemsetAsync(fail, 0, w.fail_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
         // speculative thresholds, then the exact selection for the query blocks
         // whose rows failed the check (a gated launch: the others return at once)
-        kern<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
-                                      pf_cap(s->k), scale2, buf, idx, 1, nullptr, fail, flags, nullptr, 0);
+        kern<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, qb1, s->Hq, s->W, s->k,
+                                                    s->W + s->k, pf_cap(s->k), scale2, buf, idx, 1,
+                                                    nullptr, fail, flags, nullptr, 0);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
-        kern<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, s->Hq, s->W, s->k, s->W + s->k,
-                                      pf_cap(s->k), scale2, buf, idx, 0, fail, nullptr, flags, nullptr, 0);
+        kern<<<grid, tcfa::kSelThreads, smem, st>>>(mq, mk, lse_p, s->L, qb1, s->Hq, s->W, s->k,
+                                                    s->W + s->k, pf_cap(s->k), scale2, buf, idx, 0,
+                                                    fail, nullptr, flags, nullptr, 0);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
     }
     return HS2_OK;
@@ -721,6 +726,63 @@ hs2_status hs2_select(const hs2_prefill_shape* shape, const void* q, const void*
     if (shape->d == 128)
         return run_full_select<128>(shape, q, k, nullptr, nullptr, l, idx, ws, st, flags, false, 2);
     return run_full_select<64>(shape, q, k, nullptr, nullptr, l, idx, ws, st, flags, false, 2);
+}
+
+}  // extern "C"
+
+namespace {
+// A query-row range [row0, row1) of every sequence: row0 on a 128-row query
+// block boundary, row1 on one or at L.
+bool rows_ok(const hs2_prefill_shape* s, int row0, int row1) {
+    return row0 >= 0 && row0 < row1 && row1 <= s->L && row0 % tcfa::BM == 0 &&
+           (row1 % tcfa::BM == 0 || row1 == s->L);
+}
+}  // namespace
+
+extern "C" {
+
+hs2_status hs2_full_attn_rows(const hs2_prefill_shape* shape, int row0, int row1, const void* q,
+                              const void* k, const void* v, void* o, float* lse,
+                              hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (!rows_ok(shape, row0, row1)) return HS2_ERR_INVALID_ARG;
+    if (!q || !k || !v || !o || !lse) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return HS2_ERR_INVALID_ARG;
+    if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (shape->d == 128)
+        return run_full_select<128>(shape, q, k, v, o, lse, nullptr, nullptr, st, flags, false, 1,
+                                    row0, row1);
+    return run_full_select<64>(shape, q, k, v, o, lse, nullptr, nullptr, st, flags, false, 1,
+                               row0, row1);
+}
+
+hs2_status hs2_select_rows(const hs2_prefill_shape* shape, int row0, int row1, const void* q,
+                           const void* k, const float* lse, int32_t* idx, void* workspace,
+                           size_t workspace_bytes, hs2_stream_t stream) {
+    hs2_status e = check_prefill(shape);
+    if (e != HS2_OK) return e;
+    if (!rows_ok(shape, row0, row1)) return HS2_ERR_INVALID_ARG;
+    if (!q || !k || !lse || !idx || !workspace) return HS2_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(lse) || !aligned16(idx) ||
+        !aligned16(workspace))
+        return HS2_ERR_INVALID_ARG;
+    if ((int64_t)shape->B * shape->L > 0x7fffffffLL) return HS2_ERR_UNSUPPORTED;
+    if (workspace_bytes < prefill_ws(shape).total) return HS2_ERR_WORKSPACE;
+    unsigned* flags = device_flags();
+    if (!flags) return HS2_ERR_CUDA;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    float* l = const_cast<float*>(lse);  // read only by the selection
+    if (shape->d == 128)
+        return run_full_select<128>(shape, q, k, nullptr, nullptr, l, idx, ws, st, flags, false, 2,
+                                    row0, row1);
+    return run_full_select<64>(shape, q, k, nullptr, nullptr, l, idx, ws, st, flags, false, 2,
+                               row0, row1);
 }
 
 size_t hs2_full_attn_select_blocks_workspace(const hs2_prefill_shape* shape, int block) {

@@ -54,13 +54,14 @@ struct FwdBars {
 
 constexpr int kThreads = 320;  // 10 warps
 
-// grid (ceil(L/128), Hq/2, B), 320 threads.  Query blocks run longest first.
+// grid (query blocks, Hq/2, B), 320 threads: the query blocks that end at qb_end
+// (exclusive), the longest first.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                       const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v, __nv_bfloat16* __restrict__ o,
-                      float* __restrict__ lse, int L, int Hq, float scale2,
+                      float* __restrict__ lse, int L, int qb_end, int Hq, float scale2,
                       unsigned* __restrict__ flags) {
     using F = Fwd<D>;
     extern __shared__ uint8_t smem_raw[];
@@ -68,8 +69,8 @@ prefill_fwd_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ FwdBars bars;
     const int warp = threadIdx.x >> 5, lane = lane_id();
-    const int nqb = (L + BM - 1) / BM;
-    const int qb = nqb - 1 - (int)blockIdx.x;
+    // query blocks qb_end - gridDim.x .. qb_end - 1, the longest first
+    const int qb = qb_end - 1 - (int)blockIdx.x;
     const int h0 = 2 * (int)blockIdx.y;
     const int b = blockIdx.z;
     const int n_kt = qb + 1;  // key tiles 0..qb (BN == BM)
@@ -491,7 +492,8 @@ HS2_DEV uint64_t warp_cut(uint64_t* buf, int cnt, int k, int* hist) {
     return thr;
 }
 
-// grid (ceil(L/128), B), kSelThreads threads.  wsbuf: [B*L][kSlices][cap] keys.
+// grid (query blocks, B), kSelThreads threads: the query blocks that end at qb_end
+// (exclusive), the longest first.  wsbuf: [B*L][kSlices][cap] keys.
 // BLK (the block-level selector of HySparse, the predecessor the HySparse2
 // summary ablates against in "Limits"): instead of streaming token
 // candidates, every score thread writes the attention mass of the 64-key
@@ -501,7 +503,8 @@ template <int D, bool BLK = false>
 __global__ void __launch_bounds__(kSelThreads, 1)
 prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                          const __grid_constant__ CUtensorMap map_k,
-                         const float* __restrict__ lse, int L, int Hq, int W, int kk, int S,
+                         const float* __restrict__ lse, int L, int qb_end, int Hq, int W, int kk,
+                         int S,
                          int cap, float scale2, uint64_t* __restrict__ wsbuf,
                          int32_t* __restrict__ idx, int speculate,
                          const unsigned* __restrict__ gate, unsigned* __restrict__ fail_qb,
@@ -512,8 +515,8 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     __shared__ SelBars bars;
     const int warp = threadIdx.x >> 5, lane = lane_id();
-    const int nqb = (L + BM - 1) / BM;
-    const int qb = nqb - 1 - (int)blockIdx.x;
+    const int nqb = (L + BM - 1) / BM;        // flags are indexed by absolute block
+    const int qb = qb_end - 1 - (int)blockIdx.x;  // the longest of the range first
     const int b = blockIdx.y;
     // the exact re-run only redoes the query blocks whose check failed
     if (gate != nullptr && __ldg(gate + (size_t)b * nqb + qb) == 0u) return;
