@@ -390,8 +390,8 @@ def run_ours(args, world, rank, local):
     if args.once:
         # one call of each bench entry point on the workloads, untimed (for
         # profilers), in a fixed order: full+select (pass 1, selection, gated
-        # re-run), a sparse layer, decode select (zeroing, pass 1, sketch
-        # score, sketch gather, gated fallbacks), a decode sparse layer, a
+        # re-run), a sparse layer, decode select (zeroing, pass 1, the sketch
+        # selection with its exact fallback), a decode sparse layer, a
         # second full layer with the first sparse layer's queries and the
         # overlap of the two selections, the block-level selector
         pf.full()
@@ -442,11 +442,11 @@ def run_ours(args, world, rank, local):
 
     # kernels per call: full select 3 (pass 1, pass 2 + selection, and pass 2
     # again gated: it returns at once unless a query block failed the check of
-    # its speculative thresholds); sparse 1; decode select 6 (workspace zeroing,
-    # pass 1, sketch score, sketch gather, and the exact pass 2 and gather,
-    # gated: they return at once unless a sequence overflowed the sketch
-    # candidates); decode sparse 1; stage 1; overlap 1; block selector 3
-    full_launches, dsel_launches = 3, 6
+    # its speculative thresholds); sparse 1; decode select 3 (workspace zeroing,
+    # pass 1, the sketch selection, which runs the exact fallback itself for a
+    # sequence whose candidates overflow); decode sparse 1; stage 1; overlap 1;
+    # block selector 3
+    full_launches, dsel_launches = 3, 3
 
     def launches(work):
         if isinstance(work, PrefillWork):
@@ -627,8 +627,8 @@ def run_ours(args, world, rank, local):
         "kernels": kernels,
         "gpu_launches": n_launch,
         "gpu_launches_note": f"timed step: {full_launches} full-select (1 gated re-run) + {nsp} "
-                             f"sparse + {dsel_launches} decode-select (2 of them gated "
-                             f"fallbacks) + {ndsp} decode sparse, the decode step replayed as "
+                             f"sparse + {dsel_launches} decode-select + {ndsp} decode sparse, "
+                             "the decode step replayed as "
                              "two CUDA graphs (gathered rows; rows staged once), 1 overlap + 3 "
                              "block-selector kernels; then the other workloads' calls",
         "wall_s_timed_region": round(wall, 3),

@@ -202,6 +202,32 @@ HS2_DEV uint4 ldg_nc(const void* p) {
     return r;
 }
 
+// L2 eviction-priority policies: a stream read once goes first, a small
+// intermediate the next kernel reads stays.
+HS2_DEV uint64_t l2_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+HS2_DEV uint64_t l2_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+HS2_DEV void st_hint_v2(void* p, uint2 v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.v2.u32 [%0], {%1, %2}, %3;" ::"l"(p), "r"(v.x),
+                 "r"(v.y), "l"(policy)
+                 : "memory");
+}
+// a coherent (L2) 16-byte load under a policy
+HS2_DEV uint4 ldcg_hint(const void* p, uint64_t policy) {
+    uint4 r;
+    asm volatile("ld.global.cg.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p), "l"(policy));
+    return r;
+}
+
 HS2_DEV void cp_async16(void* smem, const void* gmem, bool valid = true) {
     uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
     int n = valid ? 16 : 0;

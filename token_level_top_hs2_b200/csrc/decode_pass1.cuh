@@ -79,12 +79,12 @@ struct P1Bars {
 
 HS2_DEV void p1_issue_raw(uint8_t* st, const CUtensorMap* mk, const CUtensorMap* mv,
                           const CUtensorMap* mks, const CUtensorMap* mvs, int tok, int b,
-                          uint64_t* bar) {
+                          uint64_t* bar, uint64_t policy) {
     mbar_arrive_expect_tx(bar, 2 * (TOK * 128 + TOK * 4));
-    tma_load_3d(st + P1Layout::RAW_K, mk, 0, tok, b, bar);
-    tma_load_3d(st + P1Layout::RAW_V, mv, 0, tok, b, bar);
-    tma_load_2d(st + P1Layout::RAW_SK, mks, tok, b, bar);
-    tma_load_2d(st + P1Layout::RAW_SV, mvs, tok, b, bar);
+    tma_load_3d_hint(st + P1Layout::RAW_K, mk, 0, tok, b, bar, policy);
+    tma_load_3d_hint(st + P1Layout::RAW_V, mv, 0, tok, b, bar, policy);
+    tma_load_2d_hint(st + P1Layout::RAW_SK, mks, tok, b, bar, policy);
+    tma_load_2d_hint(st + P1Layout::RAW_SV, mvs, tok, b, bar, policy);
 }
 
 // grid (n_chunks, B), kP1Threads threads; the last chunk of a sequence to finish
@@ -159,12 +159,15 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     if (warp == kWProd) {
         if (lane == 0 && n > 0) {
             // ------------------------------------------------------ producer
+            // the cache is read once: its lines leave L2 first, so that the
+            // sketch written meanwhile stays there for the selection
+            const uint64_t pol = l2_evict_first();
             int armed = 0;
             for (int j = 0; j < n && !*abort_; j++) {
                 const int st = j % kNR, u = j / kNR;
                 if (u > 0 && !mbar_wait(&bars.raw_empty[st], (u - 1) & 1, abort_, flags)) break;
                 p1_issue_raw(smem + LY::OFF_RAW + st * LY::RAW, &map_k, &map_v, &map_ks, &map_vs,
-                             s_begin + j * TOK, b, &bars.raw_full[st]);
+                             s_begin + j * TOK, b, &bars.raw_full[st], pol);
                 armed++;
             }
             if (*abort_) {
@@ -315,6 +318,8 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         float* gred = red + g * (4 * NH);        // [4][NH]
         const int bar_vote = 1 + 2 * g, bar_red = 2 + 2 * g;
         uint8_t* pf = smem + LY::OFF_P;
+        // the sketch is read back by the next kernel: keep it in L2
+        const uint64_t sk_pol = l2_evict_last();
         // R = running max - kSk: probabilities are formed as 2^(x - R), in
         // (0, 2^(kLazy + kSk)], which is the range the sketch codes cover
         float R[NH], l[NH];
@@ -413,7 +418,7 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     for (int i = 0; i < NH / 2; i++) hw[i] = f16x2_rz(pr[2 * i], pr[2 * i + 1]);
                     const uint2 cw = make_uint2(prmt(hw[0] >> 7, hw[1] >> 7, 0x6420u),
                                                 prmt(hw[2] >> 7, hw[3] >> 7, 0x6420u));
-                    *reinterpret_cast<uint2*>(sketch + ((size_t)b * Tmax + tok) * 16 + h0) = cw;
+                    st_hint_v2(sketch + ((size_t)b * Tmax + tok) * 16 + h0, cw, sk_pol);
                 }
                 if (wq == 0 && lane < NH) {
                     float rv = R[0];
@@ -495,26 +500,50 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     __syncthreads();
     if (!bars.last) return;
     __threadfence();
+    // every chunk's maximum and sum once (the pipeline buffers are free now),
+    // then per row the merged maximum M, the chunks' factors 2^(m_i - M) and
+    // the sum; then the O sums, their loads independent of one another
     const float* pb = part + (size_t)b * n_chunks * PART;
+    float* fm = reinterpret_cast<float*>(smem);  // [n_chunks][16] m_i, then 2^(m_i - M)
+    float* fl = fm + n_chunks * 16;              // [n_chunks][16] l_i
+    float* rs = fl + n_chunks * 16;              // [16] merged sums
+    for (int i = threadIdx.x; i < n_chunks * 16; i += blockDim.x) {
+        const float* p = pb + (size_t)(i >> 4) * PART + 16 * D + (i & 15);
+        fm[i] = __ldcg(p);
+        fl[i] = __ldcg(p + 16);
+    }
+    __syncthreads();
+    if (threadIdx.x < Hq) {
+        const int row = threadIdx.x;
+        float mx = -INFINITY;
+        for (int i = 0; i < n_chunks; i++) mx = fmaxf(mx, fm[i * 16 + row]);
+        const float mu = mx == -INFINITY ? 0.f : mx;
+        float ls = 0.f;
+        for (int i = 0; i < n_chunks; i++) {
+            const float f = ex2(fm[i * 16 + row] - mu);
+            fm[i * 16 + row] = f;
+            ls += f * fl[i * 16 + row];
+        }
+        rs[row] = ls;
+        const float l2 = ls > 0.f ? mu + __log2f(ls) : -INFINITY;
+        lse2_ws[b * 16 + row] = l2;
+        if (lse_out) lse_out[b * Hq + row] = l2 * kLn2;
+    }
+    __syncthreads();
     for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
         const int row = e / D;
-        float mx = -INFINITY;
-        for (int i = 0; i < n_chunks; i++)
-            mx = fmaxf(mx, __ldcg(pb + (size_t)i * PART + 16 * D + row));
-        const float mu = mx == -INFINITY ? 0.f : mx;
-        float acc = 0.f, ls = 0.f;
-        for (int i = 0; i < n_chunks; i++) {
-            const float* p = pb + (size_t)i * PART;
-            const float f = ex2(__ldcg(p + 16 * D + row) - mu);
-            acc += f * __ldcg(p + e);
-            ls += f * __ldcg(p + 16 * D + 16 + row);
+        float acc = 0.f;
+        int i = 0;
+        for (; i + 4 <= n_chunks; i += 4) {
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) v[u] = __ldcg(pb + (size_t)(i + u) * PART + e);
+#pragma unroll
+            for (int u = 0; u < 4; u++) acc += fm[(i + u) * 16 + row] * v[u];
         }
+        for (; i < n_chunks; i++) acc += fm[i * 16 + row] * __ldcg(pb + (size_t)i * PART + e);
+        const float ls = rs[row];
         out[(size_t)b * Hq * D + e] = __float2bfloat16_rn(ls > 0.f ? acc / ls : 0.f);
-        if (e % D == 0) {
-            const float l2 = ls > 0.f ? mu + __log2f(ls) : -INFINITY;
-            lse2_ws[b * 16 + row] = l2;
-            if (lse_out) lse_out[b * Hq + row] = l2 * kLn2;
-        }
     }
 }
 

@@ -363,28 +363,24 @@ pass2_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ 
 }
 
 // ------------------------------------------------------------------ gather
-// grid (n_chunks, B), 256 threads.
+// The exact cut of one chunk (every thread of the CTA, blockDim.x >= 256):
+// the bin of the k-th largest score from the sequence's histogram; the
+// chunk's scores above it go into the row, those inside it to the boundary
+// buffer; the last CTA of the sequence adds the window, the boundary bin's
+// best keys (ties to the lower position) and the padding.  sk: BCAP keys of
+// shared memory.
 struct GatherShared {
     int bin, above, in_bin;
     unsigned last;
     int hist[260];
 };
 
-__global__ void __launch_bounds__(256)
-gather_kernel(const float* __restrict__ scores, int score_ld, const unsigned* __restrict__ hist_g,
-              const int32_t* __restrict__ lengths, int Tmax, int Hq, int W, int k,
-              int chunk_len, int n_chunks, unsigned* __restrict__ out_cnt,
-              unsigned* __restrict__ bnd_cnt, uint64_t* __restrict__ bnd,
-              unsigned* __restrict__ counter, int32_t* __restrict__ idx,
-              const unsigned* __restrict__ gate) {
-    extern __shared__ uint64_t sk[];  // BCAP keys (last CTA)
-    __shared__ GatherShared sh;
-    const int b = blockIdx.y, chunk = blockIdx.x;
-    // the scores, their histogram and the gate come from the kernels before
-    griddep_launch();
-    griddep_wait();
-    if (gate != nullptr && __ldcg(gate + b) == 0u) return;
-    const int T = __ldg(lengths + b);
+HS2_DEV void exact_gather_chunk(const float* __restrict__ scores, int score_ld,
+                                const unsigned* __restrict__ hist_g, int b, int T, int Tmax,
+                                int Hq, int W, int k, int chunk, int chunk_len, int n_chunks,
+                                unsigned* __restrict__ out_cnt, unsigned* __restrict__ bnd_cnt,
+                                uint64_t* __restrict__ bnd, unsigned* __restrict__ counter,
+                                int32_t* __restrict__ idx, uint64_t* sk, GatherShared& sh) {
     const bool ok = T >= 1 && T <= Tmax;
     const int n_cand = ok ? max(0, T - W) : 0;
     const int t = T - 1;
@@ -481,6 +477,24 @@ gather_kernel(const float* __restrict__ scores, int score_ld, const unsigned* __
     }
     __syncthreads();
     for (int i = wl + n_glob + threadIdx.x; i < S; i += blockDim.x) row[i] = -1;
+}
+
+// grid (n_chunks, B), 256 threads, dynamic shared memory BCAP keys: the exact
+// cut after the exact pass 2.
+__global__ void __launch_bounds__(256)
+gather_kernel(const float* __restrict__ scores, int score_ld, const unsigned* __restrict__ hist_g,
+              const int32_t* __restrict__ lengths, int Tmax, int Hq, int W, int k,
+              int chunk_len, int n_chunks, unsigned* __restrict__ out_cnt,
+              unsigned* __restrict__ bnd_cnt, uint64_t* __restrict__ bnd,
+              unsigned* __restrict__ counter, int32_t* __restrict__ idx) {
+    extern __shared__ uint64_t sk[];  // BCAP keys (last CTA)
+    __shared__ GatherShared sh;
+    // the scores and their histogram come from the kernel before
+    griddep_launch();
+    griddep_wait();
+    const int b = blockIdx.y;
+    exact_gather_chunk(scores, score_ld, hist_g, b, __ldg(lengths + b), Tmax, Hq, W, k, blockIdx.x,
+                       chunk_len, n_chunks, out_cnt, bnd_cnt, bnd, counter, idx, sk, sh);
 }
 
 }  // namespace dec

@@ -413,10 +413,11 @@ DecodeWs2 decode_ws2(const hs2_decode_shape* s) {
     const size_t part_floats = (size_t)16 * s->d + 32;
     size_t off = 0;
     // zeroed per call: pass-1 counter, gather counter, out count, boundary count,
-    // histogram; then the sketch selection's counter, (a spare word), boundary
-    // count, overflow flag and histogram
+    // histogram; then the sketch selection's counter, arrival counter, boundary
+    // count, overflow flag and histogram; then its verdict and the exact
+    // fallback's arrival counter
     w.zero_off = off;
-    w.zero_bytes = B * (8 + 512) * sizeof(unsigned);
+    w.zero_bytes = B * (8 + 512 + 8) * sizeof(unsigned);
     off = round_up(off + w.zero_bytes, 256);
     w.lse2_off = off;  off = round_up(off + B * 16 * sizeof(float), 256);
     w.part_off = off;  off = round_up(off + B * w.n_chunks * part_floats * sizeof(float), 256);
@@ -452,6 +453,9 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     unsigned* bnd_cnt = zero + 3 * B;
     unsigned* hist = zero + 4 * B;
     unsigned* sk_cnt = zero + 260 * B;
+    unsigned* sk_arrive = zero + 261 * B;
+    unsigned* verdict = zero + 520 * B;
+    unsigned* ex_arrive = zero + 521 * B;
     unsigned* sk_bnd = zero + 262 * B;
     unsigned* sk_ovf = zero + 263 * B;
     unsigned* sk_hist = zero + 264 * B;
@@ -460,7 +464,6 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     float* scores = reinterpret_cast<float*>(ws + w.score_off);
     uint64_t* bnd = reinterpret_cast<uint64_t*>(ws + w.bnd_off);
     const float qk_scale = s->scale * kLog2e * (FP8 ? 256.f : 1.f);
-    const unsigned* gate = nullptr;
     CUtensorMap mk, mv, mks, mvs;
     if (!map_cache(&mk, kc, s->B, s->Tmax, D, FP8) || !map_cache(&mv, vc, s->B, s->Tmax, D, FP8))
         return HS2_ERR_CUDA;
@@ -473,15 +476,23 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
     }
     const auto* qp = static_cast<const __nv_bfloat16*>(q);
     if constexpr (FP8 && D == 128) {
+        if (decode_uses_sketch(s) && w.n_chunks > 1) {
+            // the sketch selection's CTAs of a sequence wait for one another:
+            // the grid must be resident at once (one CTA per SM)
+            int dev = 0, sms = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return HS2_ERR_CUDA;
+            if ((long long)w.n_chunks * s->B > sms) return HS2_ERR_UNSUPPORTED;
+        }
         // a chain of launches with programmatic serialisation: each kernel's
         // launch and prologue overlap the tail of the one before
-        const int n16 = (int)(w.zero_bytes / 16);  // zero_bytes = B * 2080
+        const int n16 = (int)(w.zero_bytes / 16);  // zero_bytes = B * 2112
         zero16_kernel<<<(n16 + 255) / 256, 256, 0, st>>>(reinterpret_cast<uint4*>(zero), n16);
         if (launch_status() != HS2_OK) return HS2_ERR_CUDA;
         // tensor-memory path: tokens as the MMA M dimension, exact f16 K/V
         const float qk2 = s->scale * kLog2e;
         using LY = dtc::P1Layout;
-        using LY2 = dtc::Layout;
         const bool sketch = decode_uses_sketch(s);
         uint8_t* skt = sketch ? ws + w.sketch_off : nullptr;
         float* rsnap = reinterpret_cast<float*>(ws + w.rsnap_off);
@@ -492,29 +503,29 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
                        skt, rsnap, w.sk_tiles, flags) != cudaSuccess)
             return HS2_ERR_CUDA;
         if (sketch) {
-            // three resident CTAs per SM over the whole batch, one wave
-            const int g_sc = 3 * 148 / s->B > 0 ? 3 * 148 / s->B : 1;
-            if (launch_pdl(dsk::sketch_score_kernel, dim3(g_sc, s->B), dim3(dsk::kScoreThreads),
-                           0, st, skt, rsnap, w.sk_tiles, lengths, s->Tmax, s->Hq, s->W, s->k,
-                           lse2, scores, w.score_ld, sk_hist) != cudaSuccess)
-                return HS2_ERR_CUDA;
-            const size_t smem = (size_t)dec::BCAP * sizeof(uint64_t);
-            if (!set_smem(dsk::sketch_gather_kernel, smem)) return HS2_ERR_CUDA;
-            if (launch_pdl(dsk::sketch_gather_kernel, dim3(w.n_chunks, s->B),
-                           dim3(dsk::kGatherThreads), smem, st, scores, w.score_ld, sk_hist,
+            // one CTA per chunk, the grid of pass 1: a single wave, so that the
+            // CTAs of a sequence can meet after adding their histograms; the
+            // chunk's L values stay in shared memory where they fit
+            static_assert(dec::BCAP * sizeof(uint64_t) >= 256 * 32 * sizeof(unsigned),
+                          "the histogram columns share the key buffer");
+            static_assert(dec::BCAP >= dsk::kCandCap, "a CTA's keys fit the key buffer");
+            const bool lsm = dsk::select_smem_bytes(true, w.chunk_len) +
+                                 sizeof(dsk::GatherShared) <= (size_t)227 * 1024;
+            auto kern = lsm ? dsk::sketch_select_kernel<true> : dsk::sketch_select_kernel<false>;
+            const dsk::ExactArgs ex{hist, ex_arrive, out_cnt, bnd_cnt, cnt3, verdict};
+            const size_t smem = dsk::select_smem_bytes(lsm, w.chunk_len);
+            if (!set_smem(kern, smem)) return HS2_ERR_CUDA;
+            if (launch_pdl(kern, dim3(w.n_chunks, s->B), dim3(dsk::kThreads), smem, st,
+                           static_cast<const uint8_t*>(skt), static_cast<const float*>(rsnap),
+                           w.sk_tiles, scores, w.score_ld, sk_hist, sk_arrive,
                            static_cast<const uint8_t*>(kc), ks, qp, lse2, qk2, lengths, s->Tmax,
                            s->Hq, s->W, s->k, w.chunk_len, w.n_chunks, sk_bnd, bnd, sk_ovf,
-                           sk_cnt, idx) != cudaSuccess)
+                           sk_cnt, idx, ex, flags) != cudaSuccess)
                 return HS2_ERR_CUDA;
-            // sequences whose candidates overflowed: exact scores, then the exact gather
-            if (!set_smem(dtc::pass2_tc_kernel, LY2::SMEM)) return HS2_ERR_CUDA;
-            if (launch_pdl(dtc::pass2_tc_kernel, dim3(w.n_chunks, s->B), dim3(dtc::kThreads),
-                           LY2::SMEM, st, mk, mks, qp, lengths, s->Tmax, s->Hq, s->W,
-                           w.chunk_len, qk2, lse2, scores, w.score_ld, hist,
-                           static_cast<const unsigned*>(sk_ovf), flags) != cudaSuccess)
-                return HS2_ERR_CUDA;
+            // the kernel writes every row, through its exact fallback where
+            // a sequence's candidates overflow
+            return HS2_OK;
         }
-        gate = sketch ? sk_ovf : nullptr;
     } else {
         if (cudaMemsetAsync(zero, 0, w.zero_bytes, st) != cudaSuccess) return HS2_ERR_CUDA;
         auto kern = dec::pass1_kernel<D, FP8>;
@@ -538,8 +549,8 @@ hs2_status run_decode_stream(const hs2_decode_shape* s, const void* q, const voi
         // waits for the kernel before at its top, whichever path launched it
         if (launch_pdl(dec::gather_kernel, dim3(w.n_chunks, s->B), dim3(256), smem, st, scores,
                        w.score_ld, static_cast<const unsigned*>(hist), lengths, s->Tmax, s->Hq,
-                       s->W, s->k, w.chunk_len, w.n_chunks, out_cnt, bnd_cnt, bnd, cnt3, idx,
-                       gate) != cudaSuccess)
+                       s->W, s->k, w.chunk_len, w.n_chunks, out_cnt, bnd_cnt, bnd, cnt3,
+                       idx) != cudaSuccess)
             return HS2_ERR_CUDA;
     }
     return HS2_OK;
