@@ -213,6 +213,12 @@ size_t hs2_decode_select_workspace(const hs2_decode_shape* shape);
  *   idx      [B, W+k] int32   out: selection, format above
  *   workspace: >= hs2_decode_select_workspace() bytes, no initialisation
  *   needed; calls on the same workspace must not overlap in time.
+ * With the e4m3 cache at d = 128 the cache is split into chunks of whole
+ * 128-token tiles, at most one per SM (n_chunks = ceil(Tmax / chunk) with
+ * n_chunks * B <= 148), and the CTAs of a sequence wait for one another
+ * (bounded waits) in the selection: when a sequence spans several chunks the
+ * call returns HS2_ERR_UNSUPPORTED on a device with fewer SMs than
+ * n_chunks * B, before any kernel runs.
  */
 hs2_status hs2_decode_select(const hs2_decode_shape* shape, const void* q, const void* k_cache,
                              const void* v_cache, const float* k_scale, const float* v_scale,
