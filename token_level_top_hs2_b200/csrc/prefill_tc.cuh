@@ -805,14 +805,35 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
             uint32_t base = tbs[row];
 #pragma unroll
             for (int q = 1; q < kSlices; q++) base = max(base, tbs[q * 128 + row]);
-            if (speculate) {
+            // one pass over the union (loads in batches): the keys whose score
+            // bits reach `base` and the largest score bits
+            uint32_t mx = 0;
+            if (speculate || n > kk) {
+                int ge = 0;
+                for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
+                    uint64_t v[kBatch];
+#pragma unroll
+                    for (int u = 0; u < kBatch; u++) {
+                        const int i = i0 + u * 32 + lane;
+                        v[u] = i < n ? get(i) : 0;
+                    }
+#pragma unroll
+                    for (int u = 0; u < kBatch; u++) {
+                        const uint32_t sb = (uint32_t)(v[u] >> 32);
+                        if (i0 + u * 32 + lane < n) {
+                            ge += sb >= base;
+                            mx = max(mx, sb);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    ge += __shfl_xor_sync(0xffffffffu, ge, o);
+                    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                }
                 // every key whose score bits reach `base` is in the union; the
                 // row is exact iff at least min(k, candidates) of them are
-                int ge = 0;
-                for (int i = lane; i < n; i += 32) ge += (uint32_t)(get(i) >> 32) >= base;
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1) ge += __shfl_xor_sync(0xffffffffu, ge, o);
-                if (ge < min(kk, max(0, t - W + 1))) {
+                if (speculate && ge < min(kk, max(0, t - W + 1))) {
                     if (lane == 0) atomicOr(fail_qb + (size_t)b * nqb + qb, 1u);
                     continue;  // the exact re-run writes this row
                 }
@@ -833,6 +854,11 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 }
                 wp += n;
             } else {
+                // no stream was ever pruned (short rows): the union is every
+                // candidate and the histogram starts 8 octaves below the largest
+                // score, instead of at 0 where every score would clamp into the
+                // top bin
+                if (base == 0u) base = mx > (8u << 23) ? mx - (8u << 23) : 0u;
 #pragma unroll
                 for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
                 __syncwarp();
