@@ -806,8 +806,16 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
 #pragma unroll
             for (int q = 1; q < kSlices; q++) base = max(base, tbs[q * 128 + row]);
             // one pass over the union (loads in batches): the keys whose score
-            // bits reach `base` and the largest score bits
+            // bits reach `base`, the largest score bits and, when a stream was
+            // pruned (base > 0 is then the origin of the cut's histogram), the
+            // histogram relative to base
             uint32_t mx = 0;
+            const bool hist_now = base != 0u && n > kk;
+            if (hist_now) {
+#pragma unroll
+                for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
+                __syncwarp();
+            }
             if (speculate || n > kk) {
                 int ge = 0;
                 for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
@@ -823,6 +831,10 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                         if (i0 + u * 32 + lane < n) {
                             ge += sb >= base;
                             mx = max(mx, sb);
+                            if (hist_now) {
+                                const int bn = rel_bin(sb, base);
+                                if (bn >= 0) atomicAdd(&hist[bn], 1);
+                            }
                         }
                     }
                 }
@@ -858,22 +870,24 @@ prefill_select_tc_kernel(const __grid_constant__ CUtensorMap map_q,
                 // candidate and the histogram starts 8 octaves below the largest
                 // score, instead of at 0 where every score would clamp into the
                 // top bin
-                if (base == 0u) base = mx > (8u << 23) ? mx - (8u << 23) : 0u;
+                if (!hist_now) {
+                    base = mx > (8u << 23) ? mx - (8u << 23) : 0u;
 #pragma unroll
-                for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
-                __syncwarp();
-                for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
-                    uint64_t v[kBatch];
+                    for (int i = 0; i < 8; i++) hist[lane * 8 + i] = 0;
+                    __syncwarp();
+                    for (int i0 = 0; i0 < n; i0 += 32 * kBatch) {
+                        uint64_t v[kBatch];
 #pragma unroll
-                    for (int u = 0; u < kBatch; u++) {
-                        const int i = i0 + u * 32 + lane;
-                        v[u] = i < n ? get(i) : 0;
-                    }
+                        for (int u = 0; u < kBatch; u++) {
+                            const int i = i0 + u * 32 + lane;
+                            v[u] = i < n ? get(i) : 0;
+                        }
 #pragma unroll
-                    for (int u = 0; u < kBatch; u++) {
-                        const int i = i0 + u * 32 + lane;
-                        const int bn = i < n ? rel_bin((uint32_t)(v[u] >> 32), base) : -1;
-                        if (bn >= 0) atomicAdd(&hist[bn], 1);
+                        for (int u = 0; u < kBatch; u++) {
+                            const int i = i0 + u * 32 + lane;
+                            const int bn = i < n ? rel_bin((uint32_t)(v[u] >> 32), base) : -1;
+                            if (bn >= 0) atomicAdd(&hist[bn], 1);
+                        }
                     }
                 }
                 __syncwarp();
