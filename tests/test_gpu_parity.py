@@ -317,6 +317,28 @@ def test_decode_select_exact_ties_take_lower_index(cuda_lib):
         assert sorted(idx[b, W:W + k].tolist()) == list(range(k))
 
 
+def test_decode_select_every_sequence_overflows(cuda_lib):
+    """Every sequence of the batch ties everywhere, so all of them take the
+    exact fallback at once (each by all the CTAs of its chunks), with ragged
+    lengths and one sequence short enough to take every candidate."""
+    B, T, Hq, d, W, k = 5, 40000, 16, 128, 128, 1024
+    x = _decode_case("e4m3", B, T, Hq, d, W, k, [40000, 33333, 26000, 9001, 1100], seed=23)
+    for b in range(B):
+        x.k_cache[b, :] = x.k_cache[b, 7]
+        x.k_scale[b, :] = x.k_scale[b, 7]
+    o, lse, idx = run_decode(cuda_lib, x)
+    ora = oracle.decode_select(x.q, x.k_cache, x.v_cache, x.lengths, W, k, kv="e4m3",
+                               k_scale=x.k_scale, v_scale=x.v_scale, probe=idx)
+    assert max_abs(o, ora["o"]) <= TOL_E4M3
+    assert max_abs(lse, ora["lse"]) <= TOL_LSE
+    t = x.lengths.numpy().astype(np.int64) - 1
+    check_structure(idx, t, W, k)
+    check_selection(idx, ora, t, W, k)
+    for b in range(B):
+        n_glob = min(k, int(x.lengths[b]) - W)
+        assert sorted(idx[b, W:W + n_glob].tolist()) == list(range(n_glob))
+
+
 def test_decode_needles_recovered(cuda_lib):
     x = _decode_case("e4m3", 4, 65536, 16, 128, 128, 1024, seed=inputs.seed_for(4, 3))
     _, _, idx = run_decode(cuda_lib, x)
