@@ -25,8 +25,9 @@
 // every key above the bin of the k-th and ranks the keys inside that bin
 // (ties to the lower position).
 // If a sequence's candidates overflow the boundary buffer (many near-equal
-// scores, e.g. repeated keys), it is flagged and the exact pass 2 and its
-// gather run for that sequence instead (their launches are gated on the flag).
+// scores, e.g. repeated keys), the last CTA's verdict sends every CTA of
+// that sequence into the exact fallback: the exact score of every token of
+// its chunk, a histogram of them, and the exact histogram cut.
 #pragma once
 
 #include "decode_tc.cuh"
@@ -161,9 +162,11 @@ HS2_DEV void exact_fallback(float* __restrict__ lrow, int score_ld, const uint8_
 //      tile) with the expression the exact pass evaluates,
 //      sum_h 2^(<q_h, k_s> sK qk2 - lse2_h), and appended to the boundary
 //      buffer with one reservation per CTA;
-//   4. the last CTA of the sequence cuts the exact top k of those keys.
-// A wait that gives up records FLAG_TIMEOUT and flags the sequence for the
-// exact fallback, which then writes its row.
+//   4. the last CTA of the sequence checks the boundary buffer and gives the
+//      verdict the others wait for: the sketch cut (it cuts the exact top k
+//      of those keys) or, on an overflow, the exact fallback by all of them.
+// A wait that gives up records FLAG_TIMEOUT: the call then reports
+// HS2_ERR_TIMEOUT and the sequence's row is not valid.
 constexpr int kTilesInFlight = 4;
 
 inline constexpr size_t select_smem_bytes(bool lsm, int chunk_len) {
