@@ -118,7 +118,7 @@ pass1_tc_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     float* skb = reinterpret_cast<float*>(smem + LY::OFF_SC);  // [kDK][128]
     float* svb = skb + kDK * TOK;                              // [kDK][128]
     float* red = reinterpret_cast<float*>(smem + LY::OFF_RED); // [4][16]
-    // the selection kernels that follow may launch now; they wait for this
+    // the selection kernel that follows may launch now; it waits for this
     // grid to complete before reading what it writes
     griddep_launch();
 
